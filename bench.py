@@ -1,0 +1,509 @@
+#!/usr/bin/env python
+"""Benchmark of the QSA hot path on B200.
+
+Default (N=1): bf16 prefill, batch 1, seq 8192, 16 query / 2 KV heads, head_dim
+128, 4 indexer heads of dim 64, block 64, top-k 32 (+ trailing block). A step is
+one pass of the whole path (compress -> score/top-k -> sparse attention) over
+that prompt, inputs resident in HBM, L2 flushed between steps. Also measured:
+  e2e       -- the same step through qsa_forward with pinned HOST buffers, the
+               host->device copies of the inputs and the device->host read of the
+               output inside the timed region;
+  decode    -- one decode step for 64 sequences with caches of 4096..32768 tokens
+               (CUDA-graph replay, L2 flushed between steps), plus its attention
+               kernel against the HBM roofline;
+  roofline  -- the attention kernel's selected-token FLOPs over its CUDA-event time
+               against the measured bf16 tensor-core peak;
+  cpu_baseline -- the fp64 CPU oracle on a bounded random sample of query rows.
+With --gpus N under torchrun each rank runs its own replica of the workload (the
+path has no cross-sequence exchange); value = all ranks' tokens / max-over-ranks time.
+--impl reference times the oracle itself as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QSA prefill tokens/s & decode µs/step at 1 B200; % of TC / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="bf16_prefill_s8192")
+    p.add_argument("--decode-workload", default="bf16_decode_b64_l4k_32k")
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    return p.parse_args(argv)
+
+
+# --------------------------------------------------------------------------- counting
+def attended_pairs(w, inp):
+    """Exact (query, key) pairs per head summed over real query rows: each row t sees
+    min(n_c, k) whole blocks plus its trailing range of (t + 1 - n_c * B) tokens."""
+    import numpy as np
+    total = 0
+    score_pairs = 0
+    for b in range(w.batch):
+        L = int(inp["kv_len"][b])
+        q_first = int(inp["q_first"][b])
+        n_q = inp["q"].shape[1]
+        t = np.arange(max(0, q_first), min(L, q_first + n_q), dtype=np.int64)
+        n_c = (t + 1) // w.block
+        total += int((np.minimum(n_c, w.topk) * w.block + (t + 1 - n_c * w.block)).sum())
+        score_pairs += int(n_c.sum())
+    return total, score_pairs
+
+
+def real_rows(inp):
+    n = 0
+    for b in range(inp["q"].shape[0]):
+        L, qf, n_q = int(inp["kv_len"][b]), int(inp["q_first"][b]), inp["q"].shape[1]
+        n += max(0, min(L, qf + n_q) - max(0, qf))
+    return n
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {k: float(pk[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def file_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """dram bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            tab = json.load(f)
+        ent = tab[kernel_key]
+        if ent.get("source_sha") != file_sha(ent["source"]):
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"qsa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+        return False
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def cpu_oracle_rate(w, inp, seconds, seed=0):
+    """fp64 oracle over a seeded uniform sample of real query rows; rows/s == tokens/s."""
+    import numpy as np
+
+    import oracle
+    g = np.random.default_rng(seed)
+    rows_all = []
+    for b in range(w.batch):
+        L, qf, n_q = int(inp["kv_len"][b]), int(inp["q_first"][b]), inp["q"].shape[1]
+        rows_all += [(b, r) for r in range(max(0, -qf), min(n_q, L - qf))]
+
+    def run(n):
+        idx = g.choice(len(rows_all), size=min(n, len(rows_all)), replace=False)
+        by_b = {}
+        for i in idx:
+            b, r = rows_all[i]
+            by_b.setdefault(b, []).append(r)
+        t0 = time.perf_counter()
+        oracle.run(w, inp, rows={b: sorted(v) for b, v in by_b.items()})
+        return len(idx), time.perf_counter() - t0
+
+    n, dt = run(32)
+    per_row = dt / max(n, 1)
+    n_main = int(min(len(rows_all), max(32, seconds / max(per_row, 1e-6))))
+    n, dt = run(n_main)
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{n} query rows drawn uniformly (seed {seed}) from the {len(rows_all)} real rows of "
+                      f"{w.name}; fp64 C oracle, OpenMP over rows; {dt:.1f} s"}
+
+
+# --------------------------------------------------------------------------- GPU arms
+def bench_prefill(args, w, inp, dist_info):
+    import torch
+
+    from block_sparse_long_15_b200 import qsa
+    from block_sparse_long_15_b200.runner import QSAPrefill, to_device
+    dev = torch.cuda.current_device()
+    p = QSAPrefill(w, inp)
+    cfg, t, ws = p.cfg, p.t, p.ws
+    kv_cap = t["k_cache"].shape[2]
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record()
+        qsa.qsa_compress_blocks(cfg, t["ki_cache"], t["kv_start"], t["kv_len"], t["kbar_cache"])
+        if evs:
+            evs[1].record()
+        qsa.qsa_index_score_topk(cfg, t["qi"], t["kbar_cache"], t["kv_len"], t["q_first"], kv_cap,
+                                 t["sel"], ws)
+        if evs:
+            evs[2].record()
+        qsa.qsa_sparse_attn(cfg, t["q"], t["k_cache"], t["v_cache"], t["sel"], t["kv_start"], t["kv_len"],
+                            t["q_first"], t["out"], ws)
+        if evs:
+            evs[3].record()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert qsa.qsa_read_device_status(ws) == qsa.QSA_OK
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(dist_info)
+    torch.cuda.synchronize()
+    n0 = qsa.qsa_kernel_launch_count()
+    with ClockSampler(dev) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+    launches = qsa.qsa_kernel_launch_count() - n0
+    barrier(dist_info)
+    torch.cuda.synchronize()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    stage_ms = [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
+    assert qsa.qsa_read_device_status(ws) == qsa.QSA_OK
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = bench_prefill_e2e(args, w, inp, p, stream)
+    return dict(step_ms=step_ms, stage_ms=stage_ms, launches=launches, clocks=clk.summary(), e2e=e2e,
+                kernel=qsa.qsa_attn_kernel_name(cfg))
+
+
+def bench_prefill_e2e(args, w, inp, p, stream):
+    """Same step through qsa_forward with pinned host inputs/outputs, copies timed."""
+    import torch
+
+    from block_sparse_long_15_b200 import qsa
+    names = {"q": "q", "qi": "qi", "k": "k_cache", "v": "v_cache", "ki": "ki_cache",
+             "kv_start": "kv_start", "kv_len": "kv_len", "q_first": "q_first"}
+    host = {k: inp[k].contiguous().pin_memory() for k in names}
+    out_h = torch.empty(p.t["out"].shape, dtype=p.t["out"].dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for k, dst in names.items():
+            p.t[dst].copy_(host[k], non_blocking=True)
+        qsa.qsa_forward(p.cfg, qsa.QSA_PREFILL, p.t, p.ws)
+        out_h.copy_(p.t["out"], non_blocking=True)
+
+    for _ in range(max(2, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = max(5, args.steps // 2)
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for i in range(n):
+        e0[i].record()
+        step()
+        e1[i].record()
+    torch.cuda.synchronize()
+    assert qsa.qsa_read_device_status(p.ws) == qsa.QSA_OK
+    ms = statistics.mean(a.elapsed_time(b) for a, b in zip(e0, e1))
+    return dict(ms=ms, h2d=h2d, d2h=d2h)
+
+
+def decode_kernel_bytes(w, inp):
+    """Algorithmic bytes of the decode attention kernel: K and V of every attended token
+    of each KV head, the query and the output rows (bf16)."""
+    esz = 2 if w.dtype == "bf16" else 4
+    total = 0
+    for b in range(w.batch):
+        L = int(inp["kv_len"][b])
+        n_c = L // w.block
+        toks = min(n_c, w.topk) * w.block + (L - n_c * w.block)
+        total += toks * w.Hkv * w.d * esz * 2 + 2 * w.Hq * w.d * esz
+    return total
+
+
+def decode_step_bytes(w, inp):
+    """Whole decode step: attention bytes + k̄ rows scored + indexer query + appended token."""
+    esz = 2 if w.dtype == "bf16" else 4
+    total = decode_kernel_bytes(w, inp)
+    for b in range(w.batch):
+        L = int(inp["kv_len"][b])
+        total += (L // w.block) * w.di * 4 + w.Hi * w.di * esz + (2 * w.Hkv * w.d + w.di) * esz * 2
+    return total
+
+
+def bench_decode(args, wd, dist_info, peaks):
+    import torch
+
+    from block_sparse_long_15_b200 import qsa, workloads as W
+    from block_sparse_long_15_b200.runner import QSADecode
+    inp = W.make_inputs(wd)
+    d = QSADecode(wd, inp)
+    dev = torch.cuda.current_device()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        d()
+    torch.cuda.synchronize()
+    assert d.status() == qsa.QSA_OK
+    # whole step as a CUDA graph
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        d()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            d()
+    torch.cuda.synchronize()
+    n = max(20, args.steps * 5)
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        g.replay()
+    for i in range(n):
+        flush.zero_()
+        e0[i].record()
+        g.replay()
+        e1[i].record()
+    torch.cuda.synchronize()
+    step_us = statistics.median(a.elapsed_time(b) for a, b in zip(e0, e1)) * 1e3
+    # the attention kernel alone (stage call), same inputs, for its roofline
+    cfg = d.cfg
+    kv_cap = d.t["k_cache"].shape[2]
+    q_first = (d.t["kv_len"] - 1).contiguous()
+    a0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    a1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for i in range(n + args.warmup):
+        flush.zero_()
+        if i >= args.warmup:
+            a0[i - args.warmup].record()
+        qsa.qsa_sparse_attn(cfg, d.t["q"], d.t["k_cache"], d.t["v_cache"], d.t["sel"], d.t["kv_start"],
+                            d.t["kv_len"], q_first, d.t["out"], d.ws)
+        if i >= args.warmup:
+            a1[i - args.warmup].record()
+    torch.cuda.synchronize()
+    assert d.status() == qsa.QSA_OK
+    attn_us = statistics.median(a.elapsed_time(b) for a, b in zip(a0, a1)) * 1e3
+    kb = decode_kernel_bytes(wd, inp)
+    sb = decode_step_bytes(wd, inp)
+    del g
+    return {"workload": wd.name, "us_per_step": step_us, "graph": True,
+            "step_bytes": sb, "step_gbs": sb / (step_us * 1e-6) / 1e9,
+            "kernel": qsa.qsa_attn_kernel_name(cfg, qsa.QSA_DECODE),
+            "roofline": {"bound": "hbm", "achieved": kb / (attn_us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": kb / (attn_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                         "traffic": ncu_traffic("attn_decode:" + wd.name), "kernel_us": attn_us,
+                         "bytes_per_launch": kb},
+            "l2": "flushed between steps (256 MiB write)"}
+
+
+# --------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws <= 1:
+        return None
+    import torch
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    import datetime
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return {"rank": rank, "world": ws, "backend": backend}
+
+
+def barrier(info):
+    if info is None:
+        return
+    import torch.distributed as dist
+    dist.barrier()
+
+
+def max_over_ranks(x: float, info) -> float:
+    if info is None:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if info["backend"] == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(ms_per_step_rank: float, tokens_per_rank: int, info):
+    """Whole-job throughput: all ranks' tokens over the slowest rank's step time."""
+    world = 1 if info is None else info["world"]
+    ms = max_over_ranks(ms_per_step_rank, info)
+    return ms, world * tokens_per_rank / (ms * 1e-3)
+
+
+# --------------------------------------------------------------------------- main
+def main(argv=None):
+    args = parse_args(argv)
+    info = dist_setup(args)
+    rank = 0 if info is None else info["rank"]
+    n_gpus = 1 if info is None else info["world"]
+    from block_sparse_long_15_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return main_reference(args, w, info, rank, n_gpus)
+
+    import torch
+    from block_sparse_long_15_b200 import build
+    build.build()
+    peaks, peak_src = load_peaks()
+    inp = W.make_inputs(w)
+    r = bench_prefill(args, w, inp, info)
+    ms_rank = statistics.mean(r["step_ms"])
+    ms, value = aggregate(ms_rank, real_rows(inp), info)
+    pairs, score_pairs = attended_pairs(w, inp)
+    attn_flops = 4.0 * w.d * w.Hq * pairs
+    score_flops = 2.0 * w.Hi * w.di * score_pairs
+    attn_ms = statistics.mean(r["stage_ms"][2])
+    achieved = attn_flops / (attn_ms * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n_gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq, "num_attention_heads": w.Hq,
+                   "num_key_value_heads": w.Hkv, "head_dim": w.d, "indexer_n_heads": w.Hi,
+                   "indexer_head_dim": w.di, "indexer_compress_ratio": w.block,
+                   "indexer_budget": w.topk * w.block, "seed": w.seed,
+                   "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": ncu_traffic("attn_prefill:" + w.name),
+                     "peak_source": f"bf16_tflops (burst) of {peak_src}", "kernel": r["kernel"],
+                     "kernel_ms": attn_ms, "flops_per_launch": attn_flops,
+                     "stage_ms": {"compress": statistics.mean(r["stage_ms"][0]),
+                                  "score_topk": statistics.mean(r["stage_ms"][1]),
+                                  "sparse_attn": attn_ms},
+                     "score_flops_per_launch": score_flops},
+        "gpu_launches": r["launches"], "clocks": r["clocks"],
+    }
+    if r["e2e"]:
+        e = r["e2e"]
+        e_ms, e_val = aggregate(e["ms"], real_rows(inp), info)
+        out["e2e"] = {"value": e_val, "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
+                      "d2h_bytes_per_step": e["d2h"], "ms_per_step": e_ms}
+    if not args.no_decode:
+        wd = W.WORKLOADS[args.decode_workload]
+        dec = bench_decode(args, wd, info, peaks)
+        dec["us_per_step"] = max_over_ranks(dec["us_per_step"], info)
+        out["decode"] = dec
+    if rank == 0 and n_gpus == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_oracle_rate(w, inp, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if info is not None:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main_reference(args, w, info, rank, n_gpus):
+    """Reference arm: the fp64 CPU oracle, timed as it stands, on rank 0 only."""
+    if rank != 0:
+        if info is not None:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    from block_sparse_long_15_b200 import workloads as W
+    inp = W.make_inputs(w)
+    per_step_s = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_oracle_rate(w, inp, per_step_s / 4, seed=1)
+    rates = [cpu_oracle_rate(w, inp, per_step_s, seed=2 + i) for i in range(args.steps)]
+    value = statistics.mean(r["value"] for r in rates)
+    ms = 1e3 * real_rows(inp) / value
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n_gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": rates[0]["cores"], "kind": "oracle",
+                            "sample": f"each step: {rates[0]['sample']}"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    if info is not None:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,266 @@
+// Host side of the QSA C ABI (include/qsa.h): argument validation, workspace
+// sizing and kernel dispatch. Nothing here allocates device memory.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "qsa_internal.h"
+
+#include <atomic>
+
+using namespace qsa;
+
+namespace qsa {
+static std::atomic<uint64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace qsa
+
+namespace {
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Qwen4ExpTextConfig indexer fields are all-or-nothing (Usage tips: "the complete
+// set of QSA indexer fields enables sparse token selection"); QSA needs exactly one
+// indexer key head (indexer_kv_heads parameter).
+qsa_status_t resolve(const qsa_config_t *c, Dims *D) {
+  if (!c) return QSA_ERR_INVALID_ARG;
+  if (c->indexer_n_heads <= 0 || c->indexer_kv_heads <= 0 || c->indexer_head_dim <= 0 ||
+      c->indexer_budget <= 0 || c->indexer_compress_ratio <= 0)
+    return QSA_ERR_INVALID_ARG;
+  if (c->indexer_kv_heads != 1) return QSA_ERR_UNSUPPORTED;
+  if (c->num_attention_heads <= 0 || c->num_key_value_heads <= 0 ||
+      c->num_attention_heads % c->num_key_value_heads != 0)
+    return QSA_ERR_INVALID_ARG;
+  if (c->head_dim <= 0 || c->head_dim % 8 != 0 || c->indexer_head_dim % 8 != 0)
+    return QSA_ERR_INVALID_ARG;
+  if (c->dtype != QSA_DTYPE_BF16 && c->dtype != QSA_DTYPE_FP32) return QSA_ERR_INVALID_ARG;
+  if (c->indexer_budget < c->indexer_compress_ratio) return QSA_ERR_INVALID_ARG;
+  if (!(c->softmax_scale == c->softmax_scale)) return QSA_ERR_INVALID_ARG;  // NaN
+  const int G = c->num_attention_heads / c->num_key_value_heads;
+  if (c->head_dim > 256 || c->indexer_head_dim > 256 || c->indexer_n_heads > 64 || G > 32 ||
+      c->indexer_compress_ratio > 256 || c->indexer_budget / c->indexer_compress_ratio > 4096)
+    return QSA_ERR_UNSUPPORTED;
+  if (D) {
+    D->Hq = c->num_attention_heads;
+    D->Hkv = c->num_key_value_heads;
+    D->G = G;
+    D->d = c->head_dim;
+    D->Hi = c->indexer_n_heads;
+    D->di = c->indexer_head_dim;
+    D->B = c->indexer_compress_ratio;
+    D->k = c->indexer_budget / c->indexer_compress_ratio;
+    D->scale = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)c->head_dim);
+    D->bf16 = c->dtype == QSA_DTYPE_BF16;
+  }
+  return QSA_OK;
+}
+
+qsa_status_t check_sizes(const Dims &D, int batch, int n_q, int kv_cap) {
+  if (batch < 0 || n_q < 0 || kv_cap < 0) return QSA_ERR_INVALID_ARG;
+  if ((long long)kv_cap / D.B > 32768) return QSA_ERR_UNSUPPORTED;
+  return QSA_OK;
+}
+
+Seqs make_seqs(const Dims &D, const int32_t *kv_start, const int32_t *kv_len, const int32_t *q_first,
+               int batch, int n_q, int kv_cap) {
+  Seqs S;
+  S.kv_start = kv_start;
+  S.kv_len = kv_len;
+  S.q_first = q_first;
+  S.batch = batch;
+  S.n_q = n_q;
+  S.kv_cap = kv_cap;
+  S.nb_cap = kv_cap / D.B;
+  return S;
+}
+
+size_t scratch_need(const Dims &D, int mode, const Seqs &S) {
+  size_t s = 0;
+  if (mode == QSA_DECODE) {
+    if (attn_decode_supported(D)) s = attn_decode_workspace(D, S);
+  } else if (attn_tc_supported(D)) {
+    s = attn_tc_workspace(D, S);
+  }
+  return (s + 255) & ~(size_t)255;
+}
+
+qsa_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return QSA_OK;
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    return QSA_ERR_UNSUPPORTED;
+  }
+  return QSA_ERR_CUDA;
+}
+
+int *status_word(void *ws) { return (int *)ws; }
+
+qsa_status_t attn_dispatch(const Dims &D, int mode, const Seqs &S, const void *q, const void *k,
+                           const void *v, const int32_t *sel, void *out, void *ws, size_t ws_bytes,
+                           cudaStream_t st) {
+  char *scratch = (char *)ws + kStatusBytes;
+  const size_t scratch_bytes = ws_bytes - kStatusBytes;
+  if (mode == QSA_DECODE && attn_decode_supported(D))
+    return cuda_status(launch_attn_decode(D, S, q, k, v, sel, out, scratch, scratch_bytes,
+                                          status_word(ws), st));
+  if (mode == QSA_PREFILL && attn_tc_supported(D))
+    return cuda_status(
+        launch_attn_tc(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
+  return cuda_status(launch_attn_simt(D, S, q, k, v, sel, out, status_word(ws), st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t qsa_abi_version(void) { return QSA_ABI_VERSION; }
+
+uint64_t qsa_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+qsa_status_t qsa_config_validate(const qsa_config_t *cfg) { return resolve(cfg, nullptr); }
+
+int32_t qsa_topk_blocks(const qsa_config_t *cfg) {
+  Dims D;
+  return resolve(cfg, &D) == QSA_OK ? D.k : 0;
+}
+
+const char *qsa_status_string(qsa_status_t s) {
+  switch (s) {
+    case QSA_OK: return "ok";
+    case QSA_ERR_INVALID_ARG: return "invalid argument";
+    case QSA_ERR_UNSUPPORTED: return "unsupported configuration or operation";
+    case QSA_ERR_CUDA: return "CUDA error";
+    case QSA_ERR_TIMEOUT: return "device wait timed out";
+    case QSA_ERR_DEVICE_CHECK: return "device-side argument check failed";
+  }
+  return "unknown status";
+}
+
+const char *qsa_attn_kernel_name(const qsa_config_t *cfg, int32_t mode) {
+  Dims D;
+  if (resolve(cfg, &D) != QSA_OK) return "none";
+  if (mode == QSA_DECODE) return attn_decode_supported(D) ? "split-kv decode" : "simt";
+  return attn_tc_supported(D) ? "tcgen05" : "simt";
+}
+
+qsa_status_t qsa_workspace_size(const qsa_config_t *cfg, int32_t mode, int32_t batch, int32_t n_q,
+                                int32_t kv_cap, size_t *bytes) {
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if (!bytes || (mode != QSA_PREFILL && mode != QSA_DECODE)) return QSA_ERR_INVALID_ARG;
+  if ((s = check_sizes(D, batch, n_q, kv_cap)) != QSA_OK) return s;
+  Seqs S = make_seqs(D, nullptr, nullptr, nullptr, batch, n_q, kv_cap);
+  *bytes = kStatusBytes + scratch_need(D, mode, S);
+  return QSA_OK;
+}
+
+qsa_status_t qsa_compress_blocks(const qsa_config_t *cfg, const void *ki, const int32_t *kv_start,
+                                 const int32_t *kv_len, const int32_t *blocks_done, int32_t batch,
+                                 int32_t kv_cap, float *kbar, qsa_stream_t stream) {
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if ((s = check_sizes(D, batch, 1, kv_cap)) != QSA_OK) return s;
+  if (batch == 0) return QSA_OK;
+  // With kv_cap < B no block can complete: the k̄ buffer is empty and may be null.
+  if (!ki || !kv_start || !kv_len || (!kbar && kv_cap / D.B > 0)) return QSA_ERR_INVALID_ARG;
+  if (!aligned16(ki) || !aligned16(kbar)) return QSA_ERR_INVALID_ARG;
+  Seqs S = make_seqs(D, kv_start, kv_len, nullptr, batch, 0, kv_cap);
+  return cuda_status(launch_compress(D, S, ki, blocks_done, kbar, nullptr, nullptr, (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_index_score_topk(const qsa_config_t *cfg, const void *qi, const float *kbar,
+                                  const int32_t *kv_len, const int32_t *q_first, int32_t batch,
+                                  int32_t n_q, int32_t kv_cap, int32_t *sel, void *workspace,
+                                  size_t workspace_bytes, qsa_stream_t stream) {
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if ((s = check_sizes(D, batch, n_q, kv_cap)) != QSA_OK) return s;
+  if (batch == 0 || n_q == 0) return QSA_OK;
+  if (!qi || (!kbar && kv_cap / D.B > 0) || !kv_len || !q_first || !sel || !workspace)
+    return QSA_ERR_INVALID_ARG;
+  if (!aligned16(qi) || !aligned16(kbar) || !aligned16(sel) || !aligned16(workspace))
+    return QSA_ERR_INVALID_ARG;
+  if (workspace_bytes < kStatusBytes) return QSA_ERR_INVALID_ARG;
+  // Scoring reads no keys, only k̄ rows (indexed by block from the sequence start),
+  // so kv_start is not needed here.
+  Seqs S = make_seqs(D, nullptr, kv_len, q_first, batch, n_q, kv_cap);
+  return cuda_status(launch_score_topk_simt(D, S, qi, kbar, sel, status_word(workspace), (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_sparse_attn(const qsa_config_t *cfg, const void *q, const void *k, const void *v,
+                             const int32_t *sel, const int32_t *kv_start, const int32_t *kv_len,
+                             const int32_t *q_first, int32_t batch, int32_t n_q, int32_t kv_cap,
+                             void *out, void *workspace, size_t workspace_bytes,
+                             qsa_stream_t stream) {
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if ((s = check_sizes(D, batch, n_q, kv_cap)) != QSA_OK) return s;
+  if (batch == 0 || n_q == 0) return QSA_OK;
+  if (!q || !k || !v || !sel || !kv_start || !kv_len || !q_first || !out || !workspace)
+    return QSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(sel) ||
+      !aligned16(workspace))
+    return QSA_ERR_INVALID_ARG;
+  Seqs S = make_seqs(D, kv_start, kv_len, q_first, batch, n_q, kv_cap);
+  if (workspace_bytes < kStatusBytes + scratch_need(D, QSA_PREFILL, S)) return QSA_ERR_INVALID_ARG;
+  return attn_dispatch(D, QSA_PREFILL, S, q, k, v, sel, out, workspace, workspace_bytes,
+                       (cudaStream_t)stream);
+}
+
+qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensors_t *t,
+                         void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if (!t || (mode != QSA_PREFILL && mode != QSA_DECODE)) return QSA_ERR_INVALID_ARG;
+  if ((s = check_sizes(D, t->batch, t->n_q, t->kv_cap)) != QSA_OK) return s;
+  if (t->batch == 0 || t->n_q == 0) return QSA_OK;
+  if (!t->q || !t->qi || !t->k_cache || !t->v_cache || !t->ki_cache ||
+      (!t->kbar_cache && t->kv_cap / D.B > 0) ||
+      !t->kbar_blocks || !t->kv_start || !t->kv_len || !t->sel || !t->out || !workspace)
+    return QSA_ERR_INVALID_ARG;
+  if (mode == QSA_PREFILL && !t->q_first) return QSA_ERR_INVALID_ARG;
+  if (mode == QSA_DECODE && (t->n_q != 1 || !t->k_new || !t->v_new || !t->ki_new))
+    return QSA_ERR_INVALID_ARG;
+  const void *ptrs[] = {t->q, t->qi, t->k_cache, t->v_cache, t->ki_cache, t->kbar_cache, t->sel,
+                        t->out, workspace};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return QSA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int32_t *q_first = t->q_first;
+  Seqs S = make_seqs(D, t->kv_start, t->kv_len, q_first, t->batch, t->n_q, t->kv_cap);
+  if (workspace_bytes < kStatusBytes + scratch_need(D, mode, S)) return QSA_ERR_INVALID_ARG;
+  int *status = status_word(workspace);
+  if (mode == QSA_PREFILL) {
+    s = cuda_status(launch_compress(D, S, t->ki_cache, nullptr, t->kbar_cache, t->kbar_blocks,
+                                    status, st));
+  } else {
+    s = cuda_status(launch_decode_append(D, S, t->k_cache, t->v_cache, t->ki_cache, t->kbar_cache,
+                                         t->kbar_blocks, t->k_new, t->v_new, t->ki_new, status, st));
+    // The decode query sits at kv_len - 1; a null q_first tells the kernels so.
+    S.q_first = nullptr;
+  }
+  if (s != QSA_OK) return s;
+  s = cuda_status(launch_score_topk_simt(D, S, t->qi, t->kbar_cache, t->sel, status, st));
+  if (s != QSA_OK) return s;
+  return attn_dispatch(D, mode, S, t->q, t->k_cache, t->v_cache, t->sel, t->out, workspace,
+                       workspace_bytes, st);
+}
+
+qsa_status_t qsa_read_device_status(void *workspace, qsa_stream_t stream, qsa_status_t *status) {
+  if (!workspace || !status) return QSA_ERR_INVALID_ARG;
+  int h = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QSA_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return QSA_ERR_CUDA;
+  *status = (qsa_status_t)h;
+  return QSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,11 @@
+// tcgen05 prefill attention (placeholder until the tensor-core kernel lands).
+#include "qsa_internal.h"
+
+namespace qsa {
+bool attn_tc_supported(const Dims &) { return false; }
+size_t attn_tc_workspace(const Dims &, const Seqs &) { return 0; }
+cudaError_t launch_attn_tc(const Dims &, const Seqs &, const void *, const void *, const void *,
+                           const int32_t *, void *, void *, size_t, int *, cudaStream_t) {
+  return cudaErrorNotSupported;
+}
+}  // namespace qsa

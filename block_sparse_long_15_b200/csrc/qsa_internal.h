@@ -1,0 +1,113 @@
+// Internal declarations shared by the QSA CUDA translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qsa.h"
+
+namespace qsa {
+
+// Resolved problem shape (from qsa_config_t after validation).
+struct Dims {
+  int Hq, Hkv, G, d;  // G = Hq / Hkv query heads per KV head
+  int Hi, di;         // indexer heads / dim
+  int B, k;           // block size (compress ratio) and blocks kept per query
+  float scale;        // softmax scale
+  bool bf16;          // element type of q, k, v, qi, ki, out
+};
+
+// Sequence geometry of one call (all device pointers).
+struct Seqs {
+  const int32_t *kv_start, *kv_len, *q_first;
+  int batch, n_q, kv_cap;
+  int nb_cap;  // kv_cap / B: rows of kbar per sequence
+};
+
+// Workspace layout: [0, 256) status word area, then kernel scratch.
+constexpr size_t kStatusBytes = 256;
+
+__device__ __forceinline__ void record_status(int *status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// A null kv_start means every sequence starts at storage index 0; a null q_first
+// means the single query row of each sequence sits at kv_len - 1 (decode).
+__device__ __forceinline__ int seq_start(const Seqs &s, int b) { return s.kv_start ? s.kv_start[b] : 0; }
+__device__ __forceinline__ int seq_qfirst(const Seqs &s, int b) {
+  return s.q_first ? s.q_first[b] : s.kv_len[b] - 1;
+}
+
+// True when the sequence's geometry fits its buffers; records a device check otherwise.
+__device__ __forceinline__ bool seq_ok(const Seqs &s, int b, int *status) {
+  const int st = seq_start(s, b), len = s.kv_len[b];
+  const bool ok = st >= 0 && len >= 0 && (long long)st + len <= (long long)s.kv_cap;
+  if (!ok) record_status(status, QSA_ERR_DEVICE_CHECK);
+  return ok;
+}
+
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Host-side count of kernel launches issued by this library.
+void note_launch(int n = 1);
+
+// Raise a kernel's dynamic shared memory limit once (the attribute is sticky), so
+// that launches stay legal while a stream is being captured into a CUDA graph.
+template <typename K>
+cudaError_t ensure_smem(K kernel, size_t bytes) {
+  static size_t granted = 48 * 1024;
+  if (bytes <= granted) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) granted = bytes;
+  return e;
+}
+
+// ---- launches (each returns the launch error, cudaSuccess otherwise) ----
+
+// Step 1: kbar[b][j] for blocks_done[b] <= j < kv_len[b] / B; optionally records
+// kv_len[b] / B into blocks_out[b].
+cudaError_t launch_compress(const Dims &D, const Seqs &S, const void *ki, const int32_t *blocks_done,
+                            float *kbar, int32_t *blocks_out, int *status, cudaStream_t st);
+
+// Steps 2+3 (CUDA cores, fp32): scores and top-k for every query row.
+cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
+                                   int32_t *sel, int *status, cudaStream_t st);
+
+// Step 4 on CUDA cores (fp32 accumulate), any supported shape.
+cudaError_t launch_attn_simt(const Dims &D, const Seqs &S, const void *q, const void *k,
+                             const void *v, const int32_t *sel, void *out, int *status,
+                             cudaStream_t st);
+
+// Step 4 on tcgen05 tensor cores (bf16, d = 128, G divides 128); returns
+// cudaErrorNotSupported when the shape is not served.
+bool attn_tc_supported(const Dims &D);
+size_t attn_tc_workspace(const Dims &D, const Seqs &S);
+cudaError_t launch_attn_tc(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
+                           const int32_t *sel, void *out, void *scratch, size_t scratch_bytes,
+                           int *status, cudaStream_t st);
+
+// Decode prologue: append the new token, check the indexer state is in step,
+// compress a just-completed block, advance kbar_blocks.
+cudaError_t launch_decode_append(const Dims &D, const Seqs &S, void *k_cache, void *v_cache,
+                                 void *ki_cache, float *kbar, int32_t *kbar_blocks,
+                                 const void *k_new, const void *v_new, const void *ki_new,
+                                 int *status, cudaStream_t st);
+
+// Split-KV decode attention (one query per sequence), HBM-bound.
+bool attn_decode_supported(const Dims &D);
+size_t attn_decode_workspace(const Dims &D, const Seqs &S);
+cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, const void *k,
+                               const void *v, const int32_t *sel, void *out, void *scratch,
+                               size_t scratch_bytes, int *status, cudaStream_t st);
+
+}  // namespace qsa

@@ -1,0 +1,378 @@
+// CUDA-core kernels of the QSA path: block compression, fp32 scoring with exact
+// top-k selection, a CUDA-core attention kernel (fp32 config and shapes the
+// tensor-core kernel does not take) and the decode prologue.
+//
+// Definitions: Hugging Face Transformers model doc "Qwen4-Exp", intro paragraph
+// on QSA and Qwen4ExpTextConfig indexer_* parameters (see include/qsa.h).
+#include <math.h>
+
+#include "qsa_internal.h"
+
+namespace qsa {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+  return x;
+}
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// ---------------------------------------------------------------------------
+// Step 1: block compression. One warp per (sequence, block); lanes over di.
+// kbar[b][j][c] = (sum_{u<B} ki[start + jB + u][c]) / B, summed in key order.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_compress(Dims D, Seqs S, const T *__restrict__ ki, const int32_t *__restrict__ blocks_done,
+           float *__restrict__ kbar, int32_t *__restrict__ blocks_out, int *status) {
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!seq_ok(S, b, status)) return;
+  const int start = seq_start(S, b), len = S.kv_len[b];
+  const int hi = len / D.B;
+  if (blocks_out && blockIdx.x == 0 && threadIdx.x == 0) blocks_out[b] = hi;
+  const int lo = blocks_done ? max(blocks_done[b], 0) : 0;
+  for (int j = lo + blockIdx.x * 8 + warp; j < hi; j += gridDim.x * 8) {
+    const T *src = ki + ((size_t)b * S.kv_cap + start + (size_t)j * D.B) * D.di;
+    float *dst = kbar + ((size_t)b * S.nb_cap + j) * D.di;
+    for (int c = lane; c < D.di; c += 32) {
+      float acc = 0.f;
+      for (int u = 0; u < D.B; ++u) acc += to_f(src[(size_t)u * D.di + c]);
+      dst[c] = acc / (float)D.B;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Steps 2+3 on CUDA cores. A CTA holds `warps` consecutive query rows of one
+// sequence, one warp per row. Compressed keys stream through shared memory in
+// chunks of 32 blocks shared by all rows; each lane scores one block:
+//   s_j = sum_h max(0, qi[h] . kbar[j])    (fp32, dot in index order)
+// Selection is an exact radix select on the fp32 bit patterns (scores are >= +0,
+// so the bit order is the value order): the k-th largest key tau is found bit by
+// bit, then blocks with key > tau are kept together with the lowest-index blocks
+// whose key equals tau -- the (-score, index) order with ties to the lower index.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void k_score_topk_simt(Dims D, Seqs S, const T *__restrict__ qi,
+                                  const float *__restrict__ kbar, int32_t *__restrict__ sel,
+                                  int *status, int warps, int nc_cap) {
+  extern __shared__ float smem[];
+  const int HD = D.Hi * D.di;
+  float *qi_s = smem;                                  // [warps][Hi*di]
+  float *kb_s = qi_s + warps * HD;                     // [32][di+1]
+  uint32_t *sc_s = (uint32_t *)(kb_s + 32 * (D.di + 1));  // [warps][nc_cap]
+  __shared__ int s_ncmax;
+
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * warps + warp;
+  const bool ok = seq_ok(S, b, status);
+  const int len = ok ? S.kv_len[b] : 0;
+  const int t = (r < S.n_q) ? seq_qfirst(S, b) + r : -1;
+  const bool valid = ok && r < S.n_q && t >= 0 && t < len;
+  const int n_c = valid ? (t + 1) / D.B : 0;
+
+  if (threadIdx.x == 0) s_ncmax = 0;
+  if (valid) {
+    const T *src = qi + ((size_t)b * S.n_q + r) * HD;
+    for (int i = lane; i < HD; i += 32) qi_s[warp * HD + i] = to_f(src[i]);
+  }
+  __syncthreads();
+  if (lane == 0 && n_c > 0) atomicMax(&s_ncmax, n_c);
+  __syncthreads();
+  const int nc_max = s_ncmax;
+  uint32_t *keys = sc_s + (size_t)warp * nc_cap;
+
+  for (int j0 = 0; j0 < nc_max; j0 += 32) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * D.di; i += blockDim.x) {
+      const int jj = i / D.di, c = i - jj * D.di, j = j0 + jj;
+      kb_s[jj * (D.di + 1) + c] = (j < nc_max) ? kbar[((size_t)b * S.nb_cap + j) * D.di + c] : 0.f;
+    }
+    __syncthreads();
+    const int j = j0 + lane;
+    if (j < n_c) {
+      float s = 0.f;
+      const float *kr = kb_s + lane * (D.di + 1);
+      for (int h = 0; h < D.Hi; ++h) {
+        const float *qh = qi_s + warp * HD + h * D.di;
+        float dot = 0.f;
+        for (int c = 0; c < D.di; ++c) dot = fmaf(qh[c], kr[c], dot);
+        s += dot > 0.f ? dot : 0.f;
+      }
+      keys[j] = __float_as_uint(s);
+    }
+  }
+  __syncwarp();
+  if (r >= S.n_q) return;
+  int32_t *out = sel + ((size_t)b * S.n_q + r) * D.k;
+  if (!valid || n_c <= D.k) {
+    for (int i = lane; i < D.k; i += 32) out[i] = (i < n_c) ? i : -1;
+    return;
+  }
+  uint32_t prefix = 0;
+  int remaining = D.k;
+  for (int bit = 30; bit >= 0; --bit) {
+    const uint32_t want = (prefix >> bit) | 1u;
+    int cnt = 0;
+    for (int j = lane; j < n_c; j += 32) cnt += ((keys[j] >> bit) == want);
+    cnt = __reduce_add_sync(kFull, cnt);
+    if (cnt >= remaining) prefix |= (1u << bit);
+    else remaining -= cnt;
+  }
+  int base = 0, tie_base = 0;
+  const unsigned lt = lanemask_lt();
+  for (int j0 = 0; j0 < n_c; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < n_c ? keys[j] : 0u;
+    const bool gt = j < n_c && key > prefix;
+    const bool eq = j < n_c && key == prefix;
+    const unsigned eq_mask = __ballot_sync(kFull, eq);
+    const bool take = gt || (eq && tie_base + __popc(eq_mask & lt) < remaining);
+    const unsigned take_mask = __ballot_sync(kFull, take);
+    if (take) out[base + __popc(take_mask & lt)] = j;
+    base += __popc(take_mask);
+    tie_base += __popc(eq_mask);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Step 4 on CUDA cores. One CTA per (query row, KV head, sequence); one warp per
+// query head of the group. Keys stream in chunks of 32 through shared memory
+// (selected blocks in ascending order, then the trailing range); each warp keeps
+// an online softmax (running max m, sum l, fp32 output in registers).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void k_attn_simt(Dims D, Seqs S, const T *__restrict__ q, const T *__restrict__ k,
+                            const T *__restrict__ v, const int32_t *__restrict__ sel,
+                            T *__restrict__ out, int *status) {
+  extern __shared__ float smem[];
+  const int d = D.d;
+  float *q_s = smem;                 // [G][d]
+  float *k_s = q_s + D.G * d;        // [32][d+1]
+  float *v_s = k_s + 32 * (d + 1);   // [32][d]
+  const int r = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = g * D.G + warp;
+  const bool ok = seq_ok(S, b, status);
+  const int len = ok ? S.kv_len[b] : 0;
+  const int start = ok ? seq_start(S, b) : 0;
+  const int t = seq_qfirst(S, b) + r;
+  T *o_row = out + (((size_t)b * S.n_q + r) * D.Hq + h) * d;
+  if (!ok || t < 0 || t >= len) {
+    for (int c = lane; c < d; c += 32) o_row[c] = from_f<T>(0.f);
+    return;
+  }
+  const T *q_row = q + (((size_t)b * S.n_q + r) * D.Hq + h) * d;
+  for (int c = lane; c < d; c += 32) q_s[warp * d + c] = to_f(q_row[c]);
+  const size_t plane = ((size_t)b * D.Hkv + g) * S.kv_cap + start;
+  const T *kb = k + plane * d;
+  const T *vb = v + plane * d;
+  const int32_t *srow = sel + ((size_t)b * S.n_q + r) * D.k;
+  const int n_c = (t + 1) / D.B;
+
+  float m = -INFINITY, l = 0.f;
+  float o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+
+  for (int s = 0; s <= D.k; ++s) {
+    int lo, hi;
+    if (s < D.k) {
+      const int blk = srow[s];
+      if (blk < 0 || blk >= n_c) continue;
+      lo = blk * D.B;
+      hi = lo + D.B;
+    } else {
+      lo = n_c * D.B;
+      hi = t + 1;
+    }
+    for (int c0 = lo; c0 < hi; c0 += 32) {
+      const int nk = min(32, hi - c0);
+      __syncthreads();
+      for (int i = threadIdx.x; i < nk * d; i += blockDim.x) {
+        const int u = i / d, c = i - u * d;
+        k_s[u * (d + 1) + c] = to_f(kb[(size_t)(c0 + u) * d + c]);
+        v_s[u * d + c] = to_f(vb[(size_t)(c0 + u) * d + c]);
+      }
+      __syncthreads();
+      float logit = -INFINITY;
+      if (lane < nk) {
+        float dot = 0.f;
+        const float *kr = k_s + lane * (d + 1);
+        const float *qr = q_s + warp * d;
+        for (int c = 0; c < d; ++c) dot = fmaf(qr[c], kr[c], dot);
+        logit = dot * D.scale;
+      }
+      const float m_new = fmaxf(m, warp_max(logit));
+      const float corr = expf(m - m_new);
+      const float p = lane < nk ? expf(logit - m_new) : 0.f;
+      l = l * corr + warp_sum(p);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] *= corr;
+      for (int u = 0; u < nk; ++u) {
+        const float pu = __shfl_sync(kFull, p, u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (lane + 32 * i < d) o[i] = fmaf(pu, v_s[u * d + lane + 32 * i], o[i]);
+      }
+      m = m_new;
+    }
+  }
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (lane + 32 * i < d) o_row[lane + 32 * i] = from_f<T>(o[i] * inv);
+}
+
+// ---------------------------------------------------------------------------
+// Decode prologue, one CTA per sequence: check the indexer state is in step
+// with the cache (kbar_blocks == (L-1)/B; a larger value means the cache was
+// cropped, which QSA does not support), append the new token at L-1, and if
+// that completes block j = L/B - 1, compress it and advance kbar_blocks.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_decode_append(Dims D, Seqs S, T *__restrict__ k_cache, T *__restrict__ v_cache,
+                T *__restrict__ ki_cache, float *__restrict__ kbar, int32_t *__restrict__ kbar_blocks,
+                const T *__restrict__ k_new, const T *__restrict__ v_new,
+                const T *__restrict__ ki_new, int *status) {
+  const int b = blockIdx.x;
+  if (!seq_ok(S, b, status)) return;
+  const int L = S.kv_len[b], start = seq_start(S, b);
+  if (L < 1) {
+    record_status(status, QSA_ERR_DEVICE_CHECK);
+    return;
+  }
+  const int have = kbar_blocks[b], need = (L - 1) / D.B;
+  if (have != need) {
+    record_status(status, have > need ? QSA_ERR_UNSUPPORTED : QSA_ERR_DEVICE_CHECK);
+    return;
+  }
+  const size_t pos = (size_t)start + L - 1;
+  for (int i = threadIdx.x; i < D.Hkv * D.d; i += blockDim.x) {
+    const int g = i / D.d, c = i - g * D.d;
+    const size_t dst = (((size_t)b * D.Hkv + g) * S.kv_cap + pos) * D.d + c;
+    k_cache[dst] = k_new[(size_t)b * D.Hkv * D.d + i];
+    v_cache[dst] = v_new[(size_t)b * D.Hkv * D.d + i];
+  }
+  for (int c = threadIdx.x; c < D.di; c += blockDim.x)
+    ki_cache[((size_t)b * S.kv_cap + pos) * D.di + c] = ki_new[(size_t)b * D.di + c];
+  if (L % D.B != 0) return;
+  __syncthreads();
+  const int j = L / D.B - 1;
+  const T *src = ki_cache + ((size_t)b * S.kv_cap + start + (size_t)j * D.B) * D.di;
+  for (int c = threadIdx.x; c < D.di; c += blockDim.x) {
+    float acc = 0.f;
+    for (int u = 0; u < D.B; ++u) acc += to_f(src[(size_t)u * D.di + c]);
+    kbar[((size_t)b * S.nb_cap + j) * D.di + c] = acc / (float)D.B;
+  }
+  if (threadIdx.x == 0) kbar_blocks[b] = L / D.B;
+}
+
+}  // namespace
+
+cudaError_t launch_compress(const Dims &D, const Seqs &S, const void *ki, const int32_t *blocks_done,
+                            float *kbar, int32_t *blocks_out, int *status, cudaStream_t st) {
+  if (S.batch == 0) return cudaSuccess;
+  const int per_cta = 8;
+  int gx = (S.nb_cap + per_cta - 1) / per_cta;
+  gx = max(1, min(gx, 1024));
+  dim3 grid(gx, S.batch);
+  note_launch();
+  if (D.bf16)
+    k_compress<__nv_bfloat16><<<grid, 256, 0, st>>>(D, S, (const __nv_bfloat16 *)ki, blocks_done, kbar,
+                                                    blocks_out, status);
+  else
+    k_compress<float><<<grid, 256, 0, st>>>(D, S, (const float *)ki, blocks_done, kbar, blocks_out,
+                                            status);
+  return cudaGetLastError();
+}
+
+static size_t score_smem(const Dims &D, int warps, int nc_cap) {
+  return sizeof(float) * ((size_t)warps * D.Hi * D.di + 32 * (D.di + 1) + (size_t)warps * nc_cap);
+}
+
+cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
+                                   int32_t *sel, int *status, cudaStream_t st) {
+  if (S.batch == 0 || S.n_q == 0) return cudaSuccess;
+  const int nc_cap = S.nb_cap;
+  int warps = S.n_q < 8 ? S.n_q : 8;
+  const size_t limit = 200 * 1024;
+  while (warps > 1 && score_smem(D, warps, nc_cap) > limit) --warps;
+  const size_t smem = score_smem(D, warps, nc_cap);
+  if (smem > limit) return cudaErrorNotSupported;
+  dim3 grid((S.n_q + warps - 1) / warps, S.batch);
+  note_launch();
+  cudaError_t e;
+  if (D.bf16) {
+    auto kern = k_score_topk_simt<__nv_bfloat16>;
+    e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, warps * 32, smem, st>>>(D, S, (const __nv_bfloat16 *)qi, kbar, sel, status, warps, nc_cap);
+  } else {
+    auto kern = k_score_topk_simt<float>;
+    e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, warps * 32, smem, st>>>(D, S, (const float *)qi, kbar, sel, status, warps, nc_cap);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_simt(const Dims &D, const Seqs &S, const void *q, const void *k,
+                             const void *v, const int32_t *sel, void *out, int *status,
+                             cudaStream_t st) {
+  if (S.batch == 0 || S.n_q == 0) return cudaSuccess;
+  const size_t smem = sizeof(float) * ((size_t)D.G * D.d + 32 * (D.d + 1) + 32 * D.d);
+  dim3 grid(S.n_q, D.Hkv, S.batch);
+  note_launch();
+  cudaError_t e;
+  if (D.bf16) {
+    auto kern = k_attn_simt<__nv_bfloat16>;
+    e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, D.G * 32, smem, st>>>(D, S, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                       (const __nv_bfloat16 *)v, sel, (__nv_bfloat16 *)out, status);
+  } else {
+    auto kern = k_attn_simt<float>;
+    e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, D.G * 32, smem, st>>>(D, S, (const float *)q, (const float *)k, (const float *)v, sel,
+                                       (float *)out, status);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_append(const Dims &D, const Seqs &S, void *k_cache, void *v_cache,
+                                 void *ki_cache, float *kbar, int32_t *kbar_blocks,
+                                 const void *k_new, const void *v_new, const void *ki_new,
+                                 int *status, cudaStream_t st) {
+  if (S.batch == 0) return cudaSuccess;
+  note_launch();
+  if (D.bf16)
+    k_decode_append<__nv_bfloat16><<<S.batch, 256, 0, st>>>(
+        D, S, (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache, (__nv_bfloat16 *)ki_cache, kbar,
+        kbar_blocks, (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new,
+        (const __nv_bfloat16 *)ki_new, status);
+  else
+    k_decode_append<float><<<S.batch, 256, 0, st>>>(D, S, (float *)k_cache, (float *)v_cache,
+                                                    (float *)ki_cache, kbar, kbar_blocks,
+                                                    (const float *)k_new, (const float *)v_new,
+                                                    (const float *)ki_new, status);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

@@ -1,0 +1,225 @@
+"""Python binding of the QSA C ABI (include/qsa.h) -- argument marshalling only.
+
+Each function has the name of the C entry point it calls and takes torch CUDA
+tensors; it checks shapes and dtypes, passes raw device pointers and the
+current CUDA stream, and raises QSAError on a non-OK status. Every step of the
+path runs in libqsa.so; there is no fallback: if the library is missing or
+fails to load, the import of this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqsa.so")
+
+QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_CUDA, QSA_ERR_TIMEOUT, QSA_ERR_DEVICE_CHECK = range(6)
+QSA_DTYPE_BF16, QSA_DTYPE_FP32 = 0, 1
+QSA_PREFILL, QSA_DECODE = 0, 1
+
+
+class QSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class qsa_config_t(ctypes.Structure):
+    _fields_ = [("num_attention_heads", ctypes.c_int32), ("num_key_value_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("indexer_n_heads", ctypes.c_int32),
+                ("indexer_kv_heads", ctypes.c_int32), ("indexer_head_dim", ctypes.c_int32),
+                ("indexer_budget", ctypes.c_int32), ("indexer_compress_ratio", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+class qsa_tensors_t(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q", ctypes.c_int32), ("kv_cap", ctypes.c_int32),
+                ("q", ctypes.c_void_p), ("qi", ctypes.c_void_p), ("k_cache", ctypes.c_void_p),
+                ("v_cache", ctypes.c_void_p), ("ki_cache", ctypes.c_void_p),
+                ("kbar_cache", ctypes.c_void_p), ("kbar_blocks", ctypes.c_void_p),
+                ("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p), ("ki_new", ctypes.c_void_p),
+                ("kv_start", ctypes.c_void_p), ("kv_len", ctypes.c_void_p), ("q_first", ctypes.c_void_p),
+                ("sel", ctypes.c_void_p), ("out", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"QSA CUDA library not built: {LIB_PATH} is missing "
+                          "(run block_sparse_long_15_b200.build.build())")
+    L = ctypes.CDLL(LIB_PATH)
+    P, V, I, S = ctypes.POINTER, ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    cfgp = P(qsa_config_t)
+    sig = {
+        "qsa_config_validate": ([cfgp], I),
+        "qsa_topk_blocks": ([cfgp], I),
+        "qsa_status_string": ([I], ctypes.c_char_p),
+        "qsa_workspace_size": ([cfgp, I, I, I, I, P(S)], I),
+        "qsa_compress_blocks": ([cfgp, V, V, V, V, I, I, V, V], I),
+        "qsa_index_score_topk": ([cfgp, V, V, V, V, I, I, I, V, V, S, V], I),
+        "qsa_sparse_attn": ([cfgp, V, V, V, V, V, V, V, I, I, I, V, V, S, V], I),
+        "qsa_forward": ([cfgp, I, P(qsa_tensors_t), V, S, V], I),
+        "qsa_read_device_status": ([V, V, P(I)], I),
+        "qsa_abi_version": ([], I),
+        "qsa_attn_kernel_name": ([cfgp, I], ctypes.c_char_p),
+        "qsa_kernel_launch_count": ([], ctypes.c_uint64),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes, f.restype = args, res
+    return L
+
+
+_lib = _load()
+
+EXPORTED = ("qsa_config_validate", "qsa_topk_blocks", "qsa_status_string", "qsa_workspace_size",
+            "qsa_compress_blocks", "qsa_index_score_topk", "qsa_sparse_attn", "qsa_forward",
+            "qsa_read_device_status", "qsa_abi_version", "qsa_attn_kernel_name",
+            "qsa_kernel_launch_count")
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.qsa_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != QSA_OK:
+        raise QSAError(status, where)
+
+
+def make_config(Hq: int, Hkv: int, d: int, Hi: int, di: int, block: int, topk: int,
+                dtype: str = "bf16", scale: float = 0.0, indexer_kv_heads: int = 1,
+                budget: Optional[int] = None) -> qsa_config_t:
+    return qsa_config_t(Hq, Hkv, d, Hi, indexer_kv_heads, di,
+                        budget if budget is not None else topk * block, block, scale,
+                        QSA_DTYPE_BF16 if dtype == "bf16" else QSA_DTYPE_FP32)
+
+
+def config_for(w) -> qsa_config_t:
+    """Config of a workload description (fields Hq, Hkv, d, Hi, di, block, topk, dtype)."""
+    return make_config(w.Hq, w.Hkv, w.d, w.Hi, w.di, w.block, w.topk, w.dtype)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _p(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("QSA tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("QSA tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _elem(cfg: qsa_config_t) -> torch.dtype:
+    return torch.bfloat16 if cfg.dtype == QSA_DTYPE_BF16 else torch.float32
+
+
+def _want(t: torch.Tensor, dtype: torch.dtype, shape, name: str):
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+# --------------------------------------------------------------------------- entry points
+def qsa_config_validate(cfg: qsa_config_t) -> int:
+    return _lib.qsa_config_validate(ctypes.byref(cfg))
+
+
+def qsa_topk_blocks(cfg: qsa_config_t) -> int:
+    return _lib.qsa_topk_blocks(ctypes.byref(cfg))
+
+
+def qsa_abi_version() -> int:
+    return _lib.qsa_abi_version()
+
+
+def qsa_attn_kernel_name(cfg: qsa_config_t, mode: int = QSA_PREFILL) -> str:
+    return _lib.qsa_attn_kernel_name(ctypes.byref(cfg), mode).decode()
+
+
+def qsa_kernel_launch_count() -> int:
+    return _lib.qsa_kernel_launch_count()
+
+
+def qsa_workspace_size(cfg: qsa_config_t, mode: int, batch: int, n_q: int, kv_cap: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.qsa_workspace_size(ctypes.byref(cfg), mode, batch, n_q, kv_cap, ctypes.byref(out)),
+           "qsa_workspace_size")
+    return out.value
+
+
+def alloc_workspace(cfg: qsa_config_t, mode: int, batch: int, n_q: int, kv_cap: int,
+                    device=None) -> torch.Tensor:
+    """Zeroed workspace bytes (the status word must start at zero)."""
+    n = qsa_workspace_size(cfg, mode, batch, n_q, kv_cap)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def qsa_compress_blocks(cfg, ki, kv_start, kv_len, kbar, blocks_done=None, stream=None):
+    batch, kv_cap = ki.shape[0], ki.shape[1]
+    _want(ki, _elem(cfg), (batch, kv_cap, cfg.indexer_head_dim), "ki")
+    _want(kbar, torch.float32, (batch, kv_cap // cfg.indexer_compress_ratio, cfg.indexer_head_dim), "kbar")
+    _check(_lib.qsa_compress_blocks(ctypes.byref(cfg), _p(ki), _p(kv_start), _p(kv_len), _p(blocks_done),
+                                    batch, kv_cap, _p(kbar), _stream(stream)), "qsa_compress_blocks")
+
+
+def qsa_index_score_topk(cfg, qi, kbar, kv_len, q_first, kv_cap, sel, workspace, stream=None):
+    batch, n_q = qi.shape[0], qi.shape[1]
+    _want(qi, _elem(cfg), (batch, n_q, cfg.indexer_n_heads, cfg.indexer_head_dim), "qi")
+    _want(sel, torch.int32, (batch, n_q, qsa_topk_blocks(cfg)), "sel")
+    _check(_lib.qsa_index_score_topk(ctypes.byref(cfg), _p(qi), _p(kbar), _p(kv_len), _p(q_first), batch,
+                                     n_q, kv_cap, _p(sel), _p(workspace), workspace.numel(),
+                                     _stream(stream)), "qsa_index_score_topk")
+
+
+def qsa_sparse_attn(cfg, q, k, v, sel, kv_start, kv_len, q_first, out, workspace, stream=None):
+    batch, n_q = q.shape[0], q.shape[1]
+    kv_cap = k.shape[2]
+    dt = _elem(cfg)
+    _want(q, dt, (batch, n_q, cfg.num_attention_heads, cfg.head_dim), "q")
+    _want(k, dt, (batch, cfg.num_key_value_heads, kv_cap, cfg.head_dim), "k")
+    _want(v, dt, (batch, cfg.num_key_value_heads, kv_cap, cfg.head_dim), "v")
+    _want(out, dt, (batch, n_q, cfg.num_attention_heads, cfg.head_dim), "out")
+    _check(_lib.qsa_sparse_attn(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(kv_start), _p(kv_len),
+                                _p(q_first), batch, n_q, kv_cap, _p(out), _p(workspace),
+                                workspace.numel(), _stream(stream)), "qsa_sparse_attn")
+
+
+def qsa_forward(cfg, mode: int, t: Dict[str, torch.Tensor], workspace, stream=None):
+    """t: q, qi, k_cache, v_cache, ki_cache, kbar_cache, kbar_blocks, kv_start, kv_len,
+    q_first (prefill), k_new / v_new / ki_new (decode), sel, out."""
+    q = t["q"]
+    batch, n_q = q.shape[0], q.shape[1]
+    kv_cap = t["k_cache"].shape[2]
+    dt = _elem(cfg)
+    for name in ("q", "qi", "k_cache", "v_cache", "ki_cache", "out"):
+        if t[name].dtype != dt:
+            raise ValueError(f"{name}: dtype {t[name].dtype}, expected {dt}")
+    T = qsa_tensors_t(batch, n_q, kv_cap, _p(q), _p(t["qi"]), _p(t["k_cache"]), _p(t["v_cache"]),
+                      _p(t["ki_cache"]), _p(t["kbar_cache"]), _p(t["kbar_blocks"]),
+                      _p(t.get("k_new")), _p(t.get("v_new")), _p(t.get("ki_new")),
+                      _p(t["kv_start"]), _p(t["kv_len"]), _p(t.get("q_first")), _p(t["sel"]),
+                      _p(t["out"]))
+    _check(_lib.qsa_forward(ctypes.byref(cfg), mode, ctypes.byref(T), _p(workspace), workspace.numel(),
+                            _stream(stream)), "qsa_forward")
+
+
+def qsa_read_device_status(workspace: torch.Tensor, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _check(_lib.qsa_read_device_status(_p(workspace), _stream(stream), ctypes.byref(out)),
+           "qsa_read_device_status")
+    return out.value

@@ -1,0 +1,66 @@
+"""Host logic of bench.py: exact work counting (against the oracle's token sets) and
+the multi-rank aggregation (max over ranks, all ranks' tokens), run as two gloo ranks."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+import oracle
+from block_sparse_long_15_b200 import workloads as W
+
+
+def test_attended_pairs_matches_oracle_token_sets():
+    w = W.small_variant(W.WORKLOADS["bf16_prefill_varlen_b8_s16384_leftpad"], seq=600, batch=3, pad_max=200)
+    inp = W.make_inputs(w)
+    pairs, score_pairs = bench.attended_pairs(w, inp)
+    want = 0
+    want_sc = 0
+    for b in range(w.batch):
+        L = int(inp["kv_len"][b])
+        for t in range(L):
+            n_c = (t + 1) // w.block
+            sel = np.array(list(range(min(n_c, w.topk))) + [-1] * max(0, w.topk - n_c), dtype=np.int32)
+            want += len(oracle.token_set(t, w.block, sel))
+            want_sc += n_c
+    assert pairs == want and score_pairs == want_sc
+    assert bench.real_rows(inp) == int(inp["kv_len"].sum())
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    info = {"rank": rank, "world": world, "backend": "gloo"}
+    ms, value = bench.aggregate(10.0 + 5.0 * rank, 8192, info)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, ms, value))
+
+
+def test_aggregate_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, ms, value in res:
+        assert ms == 15.0  # the slowest rank's time
+        assert value == pytest.approx(2 * 8192 / 15e-3)
