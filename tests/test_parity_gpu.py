@@ -223,7 +223,8 @@ def test_decode_crop_is_rejected(cuda_lib):
     torch.cuda.synchronize()
     assert d.status() == qsa.QSA_ERR_UNSUPPORTED
     assert torch.equal(d.t["kbar_blocks"][0], before_blocks[0])
-    assert torch.equal(d.t["k_cache"][0], before_k[0])
+    # compare bit patterns: the unused cache rows hold NaN poison
+    assert torch.equal(d.t["k_cache"][0].view(torch.int16), before_k[0].view(torch.int16))
 
 
 def test_device_check_on_bad_lengths(cuda_lib):
