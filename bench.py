@@ -223,17 +223,21 @@ def bench_prefill(args, w, inp, dist_info):
     torch.cuda.synchronize()
     assert qsa.qsa_read_device_status(ws) == qsa.QSA_OK
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    barrier(dist_info)
-    torch.cuda.synchronize()
-    n0 = qsa.qsa_kernel_launch_count()
     with ClockSampler(dev) as clk:
+        # the same load before and after the timed steps, so that the 200 ms clock
+        # samples bracket the (much shorter) timed region
+        load_for(0.5, lambda: (flush.zero_(), step()))
+        barrier(dist_info)
+        torch.cuda.synchronize()
+        n0 = qsa.qsa_kernel_launch_count()
         for i in range(args.steps):
             flush.zero_()
             step(evs[i])
         torch.cuda.synchronize()
-    launches = qsa.qsa_kernel_launch_count() - n0
-    barrier(dist_info)
-    torch.cuda.synchronize()
+        launches = qsa.qsa_kernel_launch_count() - n0
+        barrier(dist_info)
+        torch.cuda.synchronize()
+        load_for(0.3, lambda: (flush.zero_(), step()))
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     stage_ms = [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
     assert qsa.qsa_read_device_status(ws) == qsa.QSA_OK
@@ -243,6 +247,16 @@ def bench_prefill(args, w, inp, dist_info):
         e2e = bench_prefill_e2e(args, w, inp, p, stream)
     return dict(step_ms=step_ms, stage_ms=stage_ms, launches=launches, clocks=clk.summary(), e2e=e2e,
                 kernel=qsa.qsa_attn_kernel_name(cfg))
+
+
+def load_for(seconds, fn):
+    """Keep the GPU busy with fn() for about `seconds` (untimed)."""
+    import torch
+    t_end = time.perf_counter() + seconds
+    while time.perf_counter() < t_end:
+        for _ in range(8):
+            fn()
+        torch.cuda.synchronize()
 
 
 def bench_prefill_e2e(args, w, inp, p, stream):
