@@ -10,9 +10,17 @@
 
 using namespace qsa;
 
+#include <stdio.h>
+
 namespace qsa {
 static std::atomic<uint64_t> g_launches{0};
+static thread_local char g_last_error[256] = "";
+static thread_local uint64_t g_error_serial = 0;
 void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+void note_error(const char *what, cudaError_t e) {
+  snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+  ++g_error_serial;
+}
 }  // namespace qsa
 
 namespace {
@@ -74,18 +82,32 @@ Seqs make_seqs(const Dims &D, const int32_t *kv_start, const int32_t *kv_len, co
   return S;
 }
 
-size_t scratch_need(const Dims &D, int mode, const Seqs &S) {
+// One query row per sequence (a decode step, or a stage call with n_q == 1) goes to
+// the split-KV decode kernel when it serves the shape; more rows go to the
+// tensor-core prefill kernel; everything else to the CUDA-core kernel.
+enum AttnKernel { kAttnSimt, kAttnTc, kAttnDecode };
+AttnKernel pick_attn(const Dims &D, const Seqs &S) {
+  if (S.n_q == 1 && attn_decode_supported(D)) return kAttnDecode;
+  if (attn_tc_supported(D)) return kAttnTc;
+  return kAttnSimt;
+}
+
+size_t scratch_need(const Dims &D, const Seqs &S) {
   size_t s = 0;
-  if (mode == QSA_DECODE) {
-    if (attn_decode_supported(D)) s = attn_decode_workspace(D, S);
-  } else if (attn_tc_supported(D)) {
-    s = attn_tc_workspace(D, S);
+  switch (pick_attn(D, S)) {
+    case kAttnDecode: s = attn_decode_workspace(D, S); break;
+    case kAttnTc: s = attn_tc_workspace(D, S); break;
+    default: break;
   }
   return (s + 255) & ~(size_t)255;
 }
 
+// Status of a launch; the launch sites record a detailed message, this records a
+// generic one only when no message was recorded since the call began.
+thread_local uint64_t g_serial_at_entry = 0;
 qsa_status_t cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return QSA_OK;
+  if (g_error_serial == g_serial_at_entry) note_error("kernel launch", e);
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
     return QSA_ERR_UNSUPPORTED;
@@ -95,18 +117,18 @@ qsa_status_t cuda_status(cudaError_t e) {
 
 int *status_word(void *ws) { return (int *)ws; }
 
-qsa_status_t attn_dispatch(const Dims &D, int mode, const Seqs &S, const void *q, const void *k,
-                           const void *v, const int32_t *sel, void *out, void *ws, size_t ws_bytes,
-                           cudaStream_t st) {
+qsa_status_t attn_dispatch(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
+                           const int32_t *sel, void *out, void *ws, size_t ws_bytes, cudaStream_t st) {
   char *scratch = (char *)ws + kStatusBytes;
   const size_t scratch_bytes = ws_bytes - kStatusBytes;
-  if (mode == QSA_DECODE && attn_decode_supported(D))
-    return cuda_status(launch_attn_decode(D, S, q, k, v, sel, out, scratch, scratch_bytes,
-                                          status_word(ws), st));
-  if (mode == QSA_PREFILL && attn_tc_supported(D))
-    return cuda_status(
-        launch_attn_tc(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
-  return cuda_status(launch_attn_simt(D, S, q, k, v, sel, out, status_word(ws), st));
+  switch (pick_attn(D, S)) {
+    case kAttnDecode:
+      return cuda_status(launch_attn_decode(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
+    case kAttnTc:
+      return cuda_status(launch_attn_tc(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
+    default:
+      return cuda_status(launch_attn_simt(D, S, q, k, v, sel, out, status_word(ws), st));
+  }
 }
 
 }  // namespace
@@ -116,6 +138,8 @@ extern "C" {
 int32_t qsa_abi_version(void) { return QSA_ABI_VERSION; }
 
 uint64_t qsa_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *qsa_last_error(void) { return g_last_error; }
 
 qsa_status_t qsa_config_validate(const qsa_config_t *cfg) { return resolve(cfg, nullptr); }
 
@@ -139,8 +163,12 @@ const char *qsa_status_string(qsa_status_t s) {
 const char *qsa_attn_kernel_name(const qsa_config_t *cfg, int32_t mode) {
   Dims D;
   if (resolve(cfg, &D) != QSA_OK) return "none";
-  if (mode == QSA_DECODE) return attn_decode_supported(D) ? "split-kv decode" : "simt";
-  return attn_tc_supported(D) ? "tcgen05" : "simt";
+  Seqs S = make_seqs(D, nullptr, nullptr, nullptr, 1, mode == QSA_DECODE ? 1 : 2, 0);
+  switch (pick_attn(D, S)) {
+    case kAttnDecode: return "split-kv decode";
+    case kAttnTc: return "tcgen05";
+    default: return "simt";
+  }
 }
 
 qsa_status_t qsa_workspace_size(const qsa_config_t *cfg, int32_t mode, int32_t batch, int32_t n_q,
@@ -151,13 +179,15 @@ qsa_status_t qsa_workspace_size(const qsa_config_t *cfg, int32_t mode, int32_t b
   if (!bytes || (mode != QSA_PREFILL && mode != QSA_DECODE)) return QSA_ERR_INVALID_ARG;
   if ((s = check_sizes(D, batch, n_q, kv_cap)) != QSA_OK) return s;
   Seqs S = make_seqs(D, nullptr, nullptr, nullptr, batch, n_q, kv_cap);
-  *bytes = kStatusBytes + scratch_need(D, mode, S);
+  if (mode == QSA_DECODE) S.n_q = 1;
+  *bytes = kStatusBytes + scratch_need(D, S);
   return QSA_OK;
 }
 
 qsa_status_t qsa_compress_blocks(const qsa_config_t *cfg, const void *ki, const int32_t *kv_start,
                                  const int32_t *kv_len, const int32_t *blocks_done, int32_t batch,
                                  int32_t kv_cap, float *kbar, qsa_stream_t stream) {
+  g_serial_at_entry = g_error_serial;
   Dims D;
   qsa_status_t s = resolve(cfg, &D);
   if (s != QSA_OK) return s;
@@ -174,6 +204,7 @@ qsa_status_t qsa_index_score_topk(const qsa_config_t *cfg, const void *qi, const
                                   const int32_t *kv_len, const int32_t *q_first, int32_t batch,
                                   int32_t n_q, int32_t kv_cap, int32_t *sel, void *workspace,
                                   size_t workspace_bytes, qsa_stream_t stream) {
+  g_serial_at_entry = g_error_serial;
   Dims D;
   qsa_status_t s = resolve(cfg, &D);
   if (s != QSA_OK) return s;
@@ -195,6 +226,7 @@ qsa_status_t qsa_sparse_attn(const qsa_config_t *cfg, const void *q, const void 
                              const int32_t *q_first, int32_t batch, int32_t n_q, int32_t kv_cap,
                              void *out, void *workspace, size_t workspace_bytes,
                              qsa_stream_t stream) {
+  g_serial_at_entry = g_error_serial;
   Dims D;
   qsa_status_t s = resolve(cfg, &D);
   if (s != QSA_OK) return s;
@@ -206,13 +238,13 @@ qsa_status_t qsa_sparse_attn(const qsa_config_t *cfg, const void *q, const void 
       !aligned16(workspace))
     return QSA_ERR_INVALID_ARG;
   Seqs S = make_seqs(D, kv_start, kv_len, q_first, batch, n_q, kv_cap);
-  if (workspace_bytes < kStatusBytes + scratch_need(D, QSA_PREFILL, S)) return QSA_ERR_INVALID_ARG;
-  return attn_dispatch(D, QSA_PREFILL, S, q, k, v, sel, out, workspace, workspace_bytes,
-                       (cudaStream_t)stream);
+  if (workspace_bytes < kStatusBytes + scratch_need(D, S)) return QSA_ERR_INVALID_ARG;
+  return attn_dispatch(D, S, q, k, v, sel, out, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensors_t *t,
                          void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+  g_serial_at_entry = g_error_serial;
   Dims D;
   qsa_status_t s = resolve(cfg, &D);
   if (s != QSA_OK) return s;
@@ -233,7 +265,7 @@ qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensor
   cudaStream_t st = (cudaStream_t)stream;
   const int32_t *q_first = t->q_first;
   Seqs S = make_seqs(D, t->kv_start, t->kv_len, q_first, t->batch, t->n_q, t->kv_cap);
-  if (workspace_bytes < kStatusBytes + scratch_need(D, mode, S)) return QSA_ERR_INVALID_ARG;
+  if (workspace_bytes < kStatusBytes + scratch_need(D, S)) return QSA_ERR_INVALID_ARG;
   int *status = status_word(workspace);
   if (mode == QSA_PREFILL) {
     s = cuda_status(launch_compress(D, S, t->ki_cache, nullptr, t->kbar_cache, t->kbar_blocks,
@@ -247,8 +279,7 @@ qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensor
   if (s != QSA_OK) return s;
   s = cuda_status(launch_score_topk_simt(D, S, t->qi, t->kbar_cache, t->sel, status, st));
   if (s != QSA_OK) return s;
-  return attn_dispatch(D, mode, S, t->q, t->k_cache, t->v_cache, t->sel, t->out, workspace,
-                       workspace_bytes, st);
+  return attn_dispatch(D, S, t->q, t->k_cache, t->v_cache, t->sel, t->out, workspace, workspace_bytes, st);
 }
 
 qsa_status_t qsa_read_device_status(void *workspace, qsa_stream_t stream, qsa_status_t *status) {

@@ -7,26 +7,27 @@
 // query rows, T = 128 / G, held as two 128-row MMA tiles A and B whose rows are
 // (token, query head of g) pairs -- the G heads that share a token's selection
 // share every K/V tile, and both tiles share every K/V chunk in shared memory.
-// The unit walks the union of its tokens' key sets in ascending 64-key chunks
-// (a chunk is one block or a part of one):
-//   warp 0      TMA producer: K and V chunks (128-byte swizzle) into two 4-deep
+// The unit walks the union of its tokens' key sets in ascending 128-key chunks
+// (two 64-key halves; a half lies inside one block):
+//   warp 0      TMA producer: K and V chunks (128-byte swizzle) into two 2-deep
 //               rings, K released after its QK MMAs, V after its PV MMAs;
-//   warp 1      TMEM owner and single-thread MMA issuer, per chunk
-//               S_A = Q_A K^T, O_A += P_A V (previous chunk), S_B = Q_B K^T,
-//               O_B += P_B V, skipping a tile for a chunk none of its rows sees;
-//               MMAs run in issue order, which orders a QK after the PV that
-//               last read the same S buffer;
+//   warp 1      TMEM owner and single-thread MMA issuer. Tiles ping-pong: for
+//               chunk i it issues O_A += P_A V_i, S_A = Q_A K_{i+1}^T, then the
+//               same for B, so one tile's softmax overlaps the other tile's MMAs.
+//               A tile with no row that sees a chunk skips it. MMAs run in issue
+//               order, which orders a QK after the PV that read the same columns;
 //   warps 2-5   softmax of tile A, warps 6-9 tile B (warp w reads TMEM lanes
-//               32 (w % 4) ..): tcgen05.ld of the S row, the row's mask (a chunk
-//               of a selected block is visible whole, a trailing chunk up to the
-//               query position, anything else not at all), online softmax with a
-//               lazily rescaled reference max, P (bf16) written back into the S
-//               columns with tcgen05.st for the PV MMA (A operand from TMEM);
-//               epilogue O / l rounded to bf16.
-// TMEM (512 columns): tile w has S buffers at 128 w + {0, 64} and O at 256 + 128 w.
+//               32 (w % 4) ..): tcgen05.ld of the 128-column S row, the row's mask
+//               per half (a half of a selected block is visible whole, a trailing
+//               half up to the query position, anything else not at all), online
+//               softmax with a lazily rescaled reference max, P (bf16) written
+//               into the first 64 S columns with tcgen05.st for the PV MMA (A
+//               operand from TMEM); epilogue O / l rounded to bf16.
+// TMEM (512 columns): S of tile w at 128 w, O of tile w at 256 + 128 w.
 // Every wait is bounded; on expiry the kernel records QSA_ERR_TIMEOUT and unwinds.
 #include <cuda.h>
 #include <math.h>
+#include <stdio.h>
 
 #include "qsa_internal.h"
 #include "sm100_ptx.cuh"
@@ -39,21 +40,24 @@ using namespace sm100;
 constexpr int kD = 128;      // head dim served
 constexpr int kRows = 128;   // MMA M: (token, head) rows per tile
 constexpr int kTiles = 2;    // tiles per CTA sharing the K/V chunks
-constexpr int kChunk = 64;   // keys per chunk (MMA N of S = Q K^T)
-constexpr int kNK = 4;       // K ring depth
-constexpr int kNV = 4;       // V ring depth
+constexpr int kChunk = 128;  // keys per chunk (MMA N of S = Q K^T, K of O += P V)
+constexpr int kHalf = 64;    // mask granularity (smallest block size served)
+constexpr int kNK = 2;       // K ring depth
+constexpr int kNV = 2;       // V ring depth
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 constexpr uint32_t kQBytes = kRows * kD * 2;    // 32 KB per tile, two 64-column halves
-constexpr uint32_t kKVBytes = kChunk * kD * 2;  // 16 KB per K (or V) chunk
+constexpr uint32_t kKVBytes = kChunk * kD * 2;  // 32 KB per K (or V) chunk, two halves
+constexpr uint32_t kSelBytes = 16384;           // selection lists of the unit, if they fit
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTiles * kQBytes;
 constexpr uint32_t kOffV = kOffK + kNK * kKVBytes;
 constexpr uint32_t kOffBar = kOffV + kNV * kKVBytes;
 constexpr uint32_t kOffMisc = kOffBar + 512;
-constexpr uint32_t kOffBitmap = kOffMisc + 64;
+constexpr uint32_t kOffSel = kOffMisc + 64;
+constexpr uint32_t kOffBitmap = kOffSel + kSelBytes;
 
 // barrier slots
 constexpr int kBarQ = 0;
@@ -61,9 +65,9 @@ constexpr int kBarKFull = 1;
 constexpr int kBarKEmpty = kBarKFull + kNK;
 constexpr int kBarVFull = kBarKEmpty + kNK;
 constexpr int kBarVEmpty = kBarVFull + kNV;
-constexpr int kBarSFull = kBarVEmpty + kNV;   // [tile][2]
-constexpr int kBarPFull = kBarSFull + 4;      // [tile][2], 4 arrivals (one per softmax warp)
-constexpr int kBarPVDone = kBarPFull + 4;     // [tile]
+constexpr int kBarSFull = kBarVEmpty + kNV;  // [tile]
+constexpr int kBarPFull = kBarSFull + 2;     // [tile], 4 arrivals (one per softmax warp)
+constexpr int kBarPVDone = kBarPFull + 2;    // [tile]
 constexpr int kNumBars = kBarPVDone + 2;
 static_assert(kNumBars * 8 <= 512, "barrier area");
 
@@ -90,12 +94,48 @@ __device__ __forceinline__ int next_chunk(const uint32_t *bm0, const uint32_t *b
   }
 }
 __device__ __forceinline__ bool bit_of(const uint32_t *bm, int c) { return (bm[c >> 5] >> (c & 31)) & 1u; }
+__device__ __forceinline__ void set_bit(uint32_t *bm, int c) { atomicOr(&bm[c >> 5], 1u << (c & 31)); }
 
 // A wait taken by a whole warp: the result is the same on every lane, so the
 // warp never splits around the warp-collective tcgen05 loads that follow.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
   const bool ok = mbar_wait(bar, parity, kWaitNs);
   return __all_sync(0xffffffffu, ok);
+}
+
+// P for one 32-key quarter, stored as 16 packed bf16 pairs at TMEM column `col`:
+// p = 2^(s * sl2 - m) for keys below `lim`, 0 from there on.
+template <bool kAll>
+__device__ __forceinline__ float p_quarter(const uint32_t *sv, int lim, float sl2, float m, uint32_t col) {
+  uint32_t pk[16];
+  float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int u = 0; u < 32; u += 2) {
+    float p0 = ex2_approx(fmaf(__uint_as_float(sv[u]), sl2, -m));
+    float p1 = ex2_approx(fmaf(__uint_as_float(sv[u + 1]), sl2, -m));
+    if (!kAll) {
+      p0 = (u < lim) ? p0 : 0.f;
+      p1 = (u + 1 < lim) ? p1 : 0.f;
+    }
+    ps[(u >> 1) & 3] += p0 + p1;
+    pk[u >> 1] = pack_bf16x2(p0, p1);
+  }
+  tmem_st16(col, pk);
+  return (ps[0] + ps[1]) + (ps[2] + ps[3]);
+}
+
+// Max of the first `lim` of 64 fp32 values, with 8 independent chains.
+template <bool kAll>
+__device__ __forceinline__ float max_half(const uint32_t *sv, int lim) {
+  float mx[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < kHalf; ++u) {
+    const float x = __uint_as_float(sv[u]);
+    mx[u & 7] = fmaxf(mx[u & 7], (kAll || u < lim) ? x : -INFINITY);
+  }
+  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -106,8 +146,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   uint64_t *bars = (uint64_t *)(base + kOffBar);
   uint32_t *tmem_slot = (uint32_t *)(base + kOffMisc);
   volatile int *abort_flag = (volatile int *)(base + kOffMisc + 8);
-  uint32_t *bmap[2] = {(uint32_t *)(base + kOffBitmap),
-                       (uint32_t *)(base + kOffBitmap) + P.bitmap_words};
+  int32_t *sel_s = (int32_t *)(base + kOffSel);
+  uint32_t *const bm0 = (uint32_t *)(base + kOffBitmap);
+  uint32_t *const bm1 = bm0 + P.bitmap_words;
 
   const Dims &D = P.D;
   const Seqs &S = P.S;
@@ -129,9 +170,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   const bool has_work = ok && r0 < S.n_q && t_lo <= t_hi;
   const int n_chunks = has_work ? t_hi / kChunk + 1 : 0;
   const int nwords = min((n_chunks + 31) >> 5, P.bitmap_words);
+  const bool sel_cached = kTiles * T * k * 4 <= (int)kSelBytes;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i >= kBarPFull && i < kBarPFull + 4) ? 4u : 1u);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 4u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -159,29 +201,27 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       tma_load_3d(&tm_q, &bars[kBarQ], dst + kQBytes / 2, 64, g * G, z);
     }
   }
-  // Per-tile chunk sets: selected blocks and trailing ranges of the tile's tokens.
+  // Per-tile chunk sets (selected blocks and trailing ranges of the tile's tokens)
+  // and a shared-memory copy of the unit's selection lists.
   if (warp >= 2 && has_work) {
     const int ts = threadIdx.x - 64;
-    for (int w = ts; w < 2 * nwords; w += 256) bmap[w / nwords][w % nwords] = 0;
+    for (int w = ts; w < 2 * nwords; w += 256) (w < nwords ? bm0 : bm1)[w % nwords] = 0;
     asm volatile("bar.sync 1, 256;" ::: "memory");
-    const int cpb = B / kChunk;
     for (int e = ts; e < kTiles * T * k; e += 256) {
       const int tok = e / k, i = e - tok * k, r = r0 + tok, t = qf + r;
       if (r >= S.n_q || t < 0 || t >= len) continue;
       const int j = P.sel[((size_t)b * S.n_q + r) * k + i];
+      if (sel_cached) sel_s[e] = j;
       if (j < 0 || j >= (t + 1) / B) continue;
-      uint32_t *bm = bmap[tok / T];
-      for (int cc = 0; cc < cpb; ++cc) {
-        const int c = j * cpb + cc;
-        atomicOr(&bm[c >> 5], 1u << (c & 31));
-      }
+      uint32_t *bm = tok < T ? bm0 : bm1;
+      for (int c = (j * B) / kChunk; c <= (j * B + B - 1) / kChunk; ++c) set_bit(bm, c);
     }
     for (int tok = ts; tok < kTiles * T; tok += 256) {
       const int r = r0 + tok, t = qf + r;
       if (r >= S.n_q || t < 0 || t >= len) continue;
-      uint32_t *bm = bmap[tok / T];
       const int lo = ((t + 1) / B) * B;
-      for (int c = lo / kChunk; lo <= t && c <= t / kChunk; ++c) atomicOr(&bm[c >> 5], 1u << (c & 31));
+      if (lo <= t)
+        for (int c = lo / kChunk; c <= t / kChunk; ++c) set_bit(tok < T ? bm0 : bm1, c);
     }
   }
   __syncthreads();
@@ -190,8 +230,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0 && has_work) {
       int i = 0;
-      for (int c = next_chunk(bmap[0], bmap[1], nwords, 0); c >= 0;
-           c = next_chunk(bmap[0], bmap[1], nwords, c + 1), ++i) {
+      for (int c = next_chunk(bm0, bm1, nwords, 0); c >= 0;
+           c = next_chunk(bm0, bm1, nwords, c + 1), ++i) {
         const int y = start + c * kChunk, z = b * D.Hkv + g;
         const int sk = i % kNK, sv = i % kNV;
         if (i >= kNK && !mbar_wait(&bars[kBarKEmpty + sk], ((i / kNK) & 1) ^ 1, kWaitNs)) {
@@ -222,78 +262,72 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, kD, false, true);
       bool fail = !mbar_wait(&bars[kBarQ], 0, kWaitNs);
       tc_fence_after();
-      int n_act[2] = {0, 0};    // chunks issued per tile
-      int pend[2] = {-1, -1};   // per-tile index of the chunk whose PV is pending
-      int v_wait_done = -1;     // union index whose V arrival has been observed
+      int n_pv0 = 0, n_pv1 = 0;  // PVs issued per tile
       auto issue_qk = [&](int w, int i) {
-        const int idx = n_act[w]++;
         const uint32_t q_addr = smem_u32(base + kOffQ + w * kQBytes);
         const uint32_t k_addr = smem_u32(base + kOffK + (i % kNK) * kKVBytes);
-        const uint32_t d_col = tbase + (uint32_t)(w * 128 + (idx & 1) * kChunk);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32;
           const uint32_t qoff = (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32;
-          mma_ss(d_col, sdesc_sw128(q_addr + qoff, 16, 1024), sdesc_sw128(k_addr + koff, 16, 1024), idesc_qk,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(tbase + (uint32_t)(w * 128), sdesc_sw128(q_addr + qoff, 16, 1024),
+                 sdesc_sw128(k_addr + koff, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[kBarSFull + w * 2 + (idx & 1)]);
-        return idx;
+        mma_commit(&bars[kBarSFull + w]);
       };
-      // PV of tile w for the chunk at union index iu (per-tile index idx).
-      auto issue_pv = [&](int w, int idx, int iu, int cu) -> bool {
-        if (!mbar_wait(&bars[kBarPFull + w * 2 + (idx & 1)], (idx >> 1) & 1, kWaitNs)) return false;
-        uint8_t *vs = base + kOffV + (iu % kNV) * kKVBytes;
-        if (v_wait_done < iu) {
-          if (!mbar_wait(&bars[kBarVFull + iu % kNV], (iu / kNV) & 1, kWaitNs)) return false;
-          v_wait_done = iu;
-          // Rows past the sequence end but inside the buffer hold whatever the cache
-          // holds there; their P is zero, but 0 * NaN is NaN, so zero them first.
-          const int valid_rows = len - cu * kChunk;
-          if (valid_rows < kChunk && start + len < S.kv_cap) {
-            for (int rr = max(valid_rows, 0); rr < kChunk; ++rr) {
-              uint4 *p0 = (uint4 *)(vs + rr * 128);
-              uint4 *p1 = (uint4 *)(vs + kKVBytes / 2 + rr * 128);
-#pragma unroll
-              for (int q = 0; q < 8; ++q) p0[q] = p1[q] = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-          }
-        }
+      auto issue_pv = [&](int w, int i) -> bool {
+        const int cnt = w ? n_pv1++ : n_pv0++;
+        if (!mbar_wait(&bars[kBarPFull + w], cnt & 1, kWaitNs)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(vs);
-        const uint32_t p_col = tbase + (uint32_t)(w * 128 + (idx & 1) * kChunk);
-        const uint32_t o_col = tbase + 256u + (uint32_t)(w * 128);
+        const uint32_t v_addr = smem_u32(base + kOffV + (i % kNV) * kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(o_col, p_col + kk * 8, sdesc_sw128(v_addr + kk * 2048, 8192, 1024), idesc_pv,
-                 (idx > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tbase + 256u + (uint32_t)(w * 128), tbase + (uint32_t)(w * 128 + kk * 8),
+                 sdesc_sw128(v_addr + kk * 2048, kKVBytes / 2, 1024), idesc_pv, (cnt > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars[kBarPVDone + w]);
         return true;
       };
-      int i = 0, c_prev = -1;
-      for (int c = next_chunk(bmap[0], bmap[1], nwords, 0); c >= 0 && !fail;
-           c = next_chunk(bmap[0], bmap[1], nwords, c + 1), ++i) {
-        const bool act[2] = {bit_of(bmap[0], c), bit_of(bmap[1], c)};
-        if (!mbar_wait(&bars[kBarKFull + i % kNK], (i / kNK) & 1, kWaitNs)) { fail = true; break; }
+      int c = next_chunk(bm0, bm1, nwords, 0);
+      if (!fail && c >= 0) {
+        if (!mbar_wait(&bars[kBarKFull], 0, kWaitNs)) fail = true;
         tc_fence_after();
-        int idx[2] = {-1, -1};
-        for (int w = 0; w < kTiles && !fail; ++w) {
-          if (act[w]) idx[w] = issue_qk(w, i);
-          if (pend[w] >= 0 && !issue_pv(w, pend[w], i - 1, c_prev)) fail = true;
+        for (int w = 0; w < kTiles && !fail; ++w)
+          if (bit_of(w ? bm1 : bm0, c)) issue_qk(w, 0);
+        mma_commit(&bars[kBarKEmpty]);
+      }
+      for (int i = 0; c >= 0 && !fail; ++i) {
+        const int c1 = next_chunk(bm0, bm1, nwords, c + 1);
+        // V of chunk i, with rows past the sequence end zeroed: their P is zero but
+        // the buffer may hold anything there, and 0 * NaN is NaN.
+        if (!mbar_wait(&bars[kBarVFull + i % kNV], (i / kNV) & 1, kWaitNs)) { fail = true; break; }
+        const int valid_rows = len - c * kChunk;
+        if (valid_rows < kChunk && start + len < S.kv_cap) {
+          uint8_t *vs = base + kOffV + (i % kNV) * kKVBytes;
+          for (int rr = max(valid_rows, 0); rr < kChunk; ++rr) {
+            uint4 *p0 = (uint4 *)(vs + rr * 128);
+            uint4 *p1 = (uint4 *)(vs + kKVBytes / 2 + rr * 128);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) p0[q] = p1[q] = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+        bool k_ready = false;
+        for (int w = 0; w < kTiles; ++w) {
+          if (bit_of(w ? bm1 : bm0, c) && !issue_pv(w, i)) { fail = true; break; }
+          if (c1 >= 0 && bit_of(w ? bm1 : bm0, c1)) {
+            if (!k_ready) {
+              if (!mbar_wait(&bars[kBarKFull + (i + 1) % kNK], ((i + 1) / kNK) & 1, kWaitNs)) { fail = true; break; }
+              tc_fence_after();
+              k_ready = true;
+            }
+            issue_qk(w, i + 1);
+          }
         }
         if (fail) break;
-        mma_commit(&bars[kBarKEmpty + i % kNK]);
-        if (i >= 1) mma_commit(&bars[kBarVEmpty + (i - 1) % kNV]);
-        pend[0] = idx[0];
-        pend[1] = idx[1];
-        c_prev = c;
+        mma_commit(&bars[kBarVEmpty + i % kNV]);
+        if (c1 >= 0) mma_commit(&bars[kBarKEmpty + (i + 1) % kNK]);
+        c = c1;
         if (*abort_flag) fail = true;
-      }
-      if (!fail && i >= 1) {
-        for (int w = 0; w < kTiles && !fail; ++w)
-          if (pend[w] >= 0 && !issue_pv(w, pend[w], i - 1, c_prev)) fail = true;
-        if (!fail) mma_commit(&bars[kBarVEmpty + (i - 1) % kNV]);
       }
       if (fail) {
         record_status(P.status, QSA_ERR_TIMEOUT);
@@ -303,109 +337,118 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
     const int w = (warp - 2) >> 2;  // tile
-    const uint32_t *bm = bmap[w];
+    const uint32_t *bm = w ? bm1 : bm0;
     const int row = 32 * (warp & 3) + lane;
     const int tok = w * T + row / G, h = row % G;
     const int r = r0 + tok, t = qf + r;
     const bool valid = has_work && r < S.n_q && t >= 0 && t < len;
     const int n_c = valid ? (t + 1) / B : 0;
-    const int32_t *srow = P.sel + ((size_t)b * S.n_q + (valid ? r : 0)) * k;
+    const int32_t *srow = sel_cached ? sel_s + tok * k : P.sel + ((size_t)b * S.n_q + (valid ? r : 0)) * k;
     const uint32_t lane_addr = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
-    const uint32_t s_col0 = lane_addr + (uint32_t)(w * 128);
+    const uint32_t s_col = lane_addr + (uint32_t)(w * 128);
     const uint32_t o_col = lane_addr + 256u + (uint32_t)(w * 128);
-    uint64_t *s_full = &bars[kBarSFull + w * 2];
-    uint64_t *p_full = &bars[kBarPFull + w * 2];
-    uint64_t *pv_done = &bars[kBarPVDone + w];
     const float sl2 = D.scale * 1.4426950408889634f;
     float m_ref = -INFINITY, l = 0.f;
     int ptr = 0, n = 0;
     bool fail = false;
     if (has_work) {
-      for (int c = next_chunk(bmap[0], bmap[1], nwords, 0); c >= 0;
-           c = next_chunk(bmap[0], bmap[1], nwords, c + 1)) {
+      for (int c = next_chunk(bm0, bm1, nwords, 0); c >= 0;
+           c = next_chunk(bm0, bm1, nwords, c + 1)) {
         if (!bit_of(bm, c)) continue;
-        const int sb = n & 1;
-        int lim = 0;
+        int lim[2] = {0, 0};
         if (valid) {
-          const int jb = (c * kChunk) / B;
-          if (jb < n_c) {
-            while (ptr < k && srow[ptr] >= 0 && srow[ptr] < jb) ++ptr;
-            lim = (ptr < k && srow[ptr] == jb) ? kChunk : 0;
-          } else {
-            const int last = t - c * kChunk;
-            lim = last >= 0 ? min(last + 1, kChunk) : 0;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int key0 = c * kChunk + hh * kHalf;
+            const int jb = key0 / B;
+            if (jb < n_c) {
+              while (ptr < k && srow[ptr] >= 0 && srow[ptr] < jb) ++ptr;
+              lim[hh] = (ptr < k && srow[ptr] == jb) ? kHalf : 0;
+            } else {
+              const int last = t - key0;
+              lim[hh] = last >= 0 ? min(last + 1, kHalf) : 0;
+            }
           }
         }
-        if (!warp_wait(&s_full[sb], (n >> 1) & 1)) { fail = true; break; }
+        const bool z0 = __all_sync(0xffffffffu, lim[0] == 0);
+        const bool z1 = __all_sync(0xffffffffu, lim[1] == 0);
+        const bool f0 = __all_sync(0xffffffffu, lim[0] == kHalf);
+        const bool f1 = __all_sync(0xffffffffu, lim[1] == kHalf);
+        if (!warp_wait(&bars[kBarSFull + w], n & 1)) { fail = true; break; }
         tc_fence_after();
-        uint32_t pk[32];
-        if (__all_sync(0xffffffffu, lim == 0)) {
+        if (z0 && z1) {
+          uint32_t zk[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) pk[q] = 0u;
+          for (int q = 0; q < 32; ++q) zk[q] = 0u;
+          tmem_st32(s_col, zk);
+          tmem_st32(s_col + 32, zk);
         } else {
-          uint32_t sv[64];
-          tmem_ld32(s_col0 + sb * kChunk, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(s_col0 + sb * kChunk + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          uint32_t sv[128];
+          if (!z0) {
+            tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          }
+          if (!z1) {
+            tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+            tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+          }
           tmem_ld_wait();
           float cmax = -INFINITY;
-#pragma unroll
-          for (int u = 0; u < 64; ++u)
-            if (u < lim) cmax = fmaxf(cmax, __uint_as_float(sv[u]));
+          if (!z0) cmax = f0 ? max_half<true>(&sv[0], kHalf) : max_half<false>(&sv[0], lim[0]);
+          if (!z1) cmax = fmaxf(cmax, f1 ? max_half<true>(&sv[kHalf], kHalf) : max_half<false>(&sv[kHalf], lim[1]));
           cmax *= sl2;
           bool rescale = false;
           float alpha = 1.f;
-          if (lim > 0) {
+          if (lim[0] > 0 || lim[1] > 0) {
             if (m_ref == -INFINITY) {
               m_ref = cmax;
             } else if (cmax > m_ref + 8.f) {
               rescale = true;
               alpha = ex2_approx(m_ref - cmax);
-            }
-          }
-          if (__any_sync(0xffffffffu, rescale)) {
-            // O is stable once PV of this tile's previous chunk has completed.
-            if (n >= 1 && !warp_wait(pv_done, (n - 1) & 1)) { fail = true; break; }
-            tc_fence_after();
-#pragma unroll 1
-            for (int cb = 0; cb < kD / 32; ++cb) {
-              uint32_t ov[32];
-              tmem_ld32(o_col + cb * 32, ov);
-              tmem_ld_wait();
-#pragma unroll
-              for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
-              tmem_st32(o_col + cb * 32, ov);
-            }
-            tmem_st_wait();
-            if (rescale) {
-              l *= alpha;
               m_ref = cmax;
             }
           }
+          // P of keys 32 q .. 32 q + 31 -> columns 16 q .. 16 q + 15.
           float psum = 0.f;
-          if (__all_sync(0xffffffffu, lim == kChunk)) {
 #pragma unroll
-            for (int u = 0; u < 64; u += 2) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(sv[u]), sl2, -m_ref));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(sv[u + 1]), sl2, -m_ref));
-              psum += p0 + p1;
-              pk[u >> 1] = pack_bf16x2(p0, p1);
-            }
-          } else {
+          for (int q = 0; q < 4; ++q) {
+            const int hh = q >> 1;
+            const int lq = lim[hh] - (q & 1) * 32;  // keys of this quarter below the limit
+            const bool zero = hh ? z1 : z0, full = hh ? f1 : f0;
+            if (zero) {
+              uint32_t zk[16];
 #pragma unroll
-            for (int u = 0; u < 64; u += 2) {
-              const float p0 = (u < lim) ? ex2_approx(fmaf(__uint_as_float(sv[u]), sl2, -m_ref)) : 0.f;
-              const float p1 = (u + 1 < lim) ? ex2_approx(fmaf(__uint_as_float(sv[u + 1]), sl2, -m_ref)) : 0.f;
-              psum += p0 + p1;
-              pk[u >> 1] = pack_bf16x2(p0, p1);
+              for (int e = 0; e < 16; ++e) zk[e] = 0u;
+              tmem_st16(s_col + 16 * q, zk);
+            } else if (full) {
+              psum += p_quarter<true>(&sv[32 * q], 32, sl2, m_ref, s_col + 16 * q);
+            } else {
+              psum += p_quarter<false>(&sv[32 * q], lq, sl2, m_ref, s_col + 16 * q);
             }
+          }
+          if (__any_sync(0xffffffffu, rescale)) {
+            // The reference max moved up: scale this row's O (and l) by alpha. O is
+            // stable once this tile's previous PV has completed, and the next PV
+            // waits for this warp's arrival below.
+            if (n >= 1 && !warp_wait(&bars[kBarPVDone + w], (n - 1) & 1)) { fail = true; break; }
+            tc_fence_after();
+#pragma unroll 1
+            for (int cb = 0; cb < kD / 16; ++cb) {
+              uint32_t ov[16];
+              tmem_ld16(o_col + cb * 16, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int q = 0; q < 16; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
+              tmem_st16(o_col + cb * 16, ov);
+            }
+            l *= alpha;
           }
           l += psum;
         }
-        tmem_st32(s_col0 + sb * kChunk, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[sb]);
+        if (lane == 0) mbar_arrive(&bars[kBarPFull + w]);
         ++n;
         if (*abort_flag) { fail = true; break; }
       }
@@ -415,7 +458,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       *abort_flag = 1;
     }
     // ---------------------------------------------------------------- epilogue
-    const bool have_o = has_work && n > 0 && !fail && warp_wait(pv_done, (n - 1) & 1);
+    const bool have_o = has_work && n > 0 && !fail && warp_wait(&bars[kBarPVDone + w], (n - 1) & 1);
     if (has_work && n > 0 && !fail && !have_o) {
       record_status(P.status, QSA_ERR_TIMEOUT);
       *abort_flag = 1;
@@ -432,18 +475,18 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       }
     } else {
 #pragma unroll 1
-      for (int cb = 0; cb < kD / 32; ++cb) {
-        uint32_t ov[32];
-        tmem_ld32(o_col + cb * 32, ov);
+      for (int cb = 0; cb < kD / 16; ++cb) {
+        uint32_t ov[16];
+        tmem_ld16(o_col + cb * 16, ov);
         tmem_ld_wait();
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
+        for (int q = 0; q < 8; ++q)
           pk[q] = pack_bf16x2(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv);
         if (write) {
-          uint4 *o4 = (uint4 *)(orow + cb * 32);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) o4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          uint4 *o4 = (uint4 *)(orow + cb * 16);
+          o4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          o4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
     }
@@ -491,7 +534,7 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_
 }  // namespace
 
 bool attn_tc_supported(const Dims &D) {
-  return D.bf16 && D.d == kD && D.G >= 1 && kRows % D.G == 0 && D.B % kChunk == 0;
+  return D.bf16 && D.d == kD && D.G >= 1 && kRows % D.G == 0 && D.B % kHalf == 0;
 }
 
 size_t attn_tc_workspace(const Dims &, const Seqs &) { return 0; }
@@ -503,6 +546,10 @@ cudaError_t launch_attn_tc(const Dims &D, const Seqs &S, const void *q, const vo
   CUtensorMap tq, tk, tv;
   const uint64_t rows_q = (uint64_t)S.batch * S.n_q;
   const int T = kRows / D.G;
+  if (!encode_fn()) {
+    note_error("cuTensorMapEncodeTiled entry point", cudaErrorNotSupported);
+    return cudaErrorNotSupported;
+  }
   if (!make_map(&tq, q, kD, D.Hq, rows_q, (uint64_t)kD * 2, (uint64_t)D.Hq * kD * 2, 64, D.G, T) ||
       !make_map(&tk, k, kD, S.kv_cap, (uint64_t)S.batch * D.Hkv, (uint64_t)kD * 2, (uint64_t)S.kv_cap * kD * 2,
                 64, kChunk, 1) ||
@@ -527,7 +574,18 @@ cudaError_t launch_attn_tc(const Dims &D, const Seqs &S, const void *q, const vo
   if (units > 0x7fffffffLL) return cudaErrorNotSupported;
   note_launch();
   k_attn_tc<<<(unsigned)units, kThreads, smem, st>>>(tq, tk, tv, P);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    cudaFuncAttributes a;
+    char what[160];
+    if (cudaFuncGetAttributes(&a, k_attn_tc) == cudaSuccess)
+      snprintf(what, sizeof what, "k_attn_tc launch (regs %d, max threads %d, smem %zu)", a.numRegs,
+               a.maxThreadsPerBlock, smem);
+    else
+      snprintf(what, sizeof what, "k_attn_tc launch");
+    note_error(what, e);
+  }
+  return e;
 }
 
 }  // namespace qsa

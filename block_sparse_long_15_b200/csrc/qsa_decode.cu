@@ -1,11 +1,369 @@
-// Split-KV decode attention (placeholder until the decode kernel lands).
+// Step 4 for decode (one query row per sequence): split-KV attention over the
+// selected blocks plus the trailing block, bound by HBM bandwidth (Hugging Face
+// Transformers model doc "Qwen4-Exp": intro paragraph on QSA; cached generation in
+// the Usage tips; GQA per Qwen4ExpTextConfig num_key_value_heads).
+//
+// The attended tokens of one (sequence, KV head) are its selected blocks (ascending)
+// followed by the trailing block. They are cut into splits of kItems blocks; one
+// CTA per (split, KV head, sequence) pulls its K and V blocks with TMA (a block of
+// one head is a contiguous 64 x 128 bf16 tile, loaded as two 128-byte-swizzled
+// boxes) into shared memory, all at once, and four warps run the G query heads of
+// the group against them with warp-level bf16 MMAs (m16n8k16: heads as rows, keys
+// as columns, fp32 accumulate) and an online softmax per warp. The warps merge in
+// shared memory and the CTA writes an fp32 partial (m, l, O) to the workspace; a
+// second kernel merges the splits of each head with the log-sum-exp rule and
+// writes bf16. Rows of a partial block beyond the sequence end are masked in S and
+// zeroed in V before use (the cache may hold anything there).
+#include <cuda.h>
+#include <math.h>
+#include <stdio.h>
+
 #include "qsa_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace qsa {
-bool attn_decode_supported(const Dims &) { return false; }
-size_t attn_decode_workspace(const Dims &, const Seqs &) { return 0; }
-cudaError_t launch_attn_decode(const Dims &, const Seqs &, const void *, const void *, const void *,
-                               const int32_t *, void *, void *, size_t, int *, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kBlk = 64;          // keys per block tile (the block size served)
+constexpr int kItems = 2;         // blocks per split
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr uint32_t kTileBytes = kBlk * kD * 2;  // 16 KB per K (or V) block
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kMaxG = 8;          // query heads per KV head served (MMA rows 0..7)
+
+struct DecParams {
+  Dims D;
+  Seqs S;
+  const __nv_bfloat16 *q;
+  const int32_t *sel;
+  __nv_bfloat16 *out;
+  float *part;      // [batch][Hkv][max_splits][G][d + 2]: O (unnormalised), m, l
+  int max_splits;
+  int *status;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
 }
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte offset of (row, 16-byte chunk) inside a 128-byte-swizzled tile of 128-byte rows.
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_attn_decode(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, DecParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *ks = base;                                  // kItems x 16 KB
+  uint8_t *vs = base + kItems * kTileBytes;            // kItems x 16 KB
+  uint64_t *bars = (uint64_t *)(base + 2 * kItems * kTileBytes);
+  float *red = (float *)(base + 2 * kItems * kTileBytes + 64);  // merge scratch
+
+  const Dims &D = P.D;
+  const Seqs &S = P.S;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool ok = seq_ok(S, b, threadIdx.x == 0 ? P.status : nullptr);
+  const int len = ok ? S.kv_len[b] : 0;
+  const int start = ok ? seq_start(S, b) : 0;
+  const int t = seq_qfirst(S, b);
+  if (!ok || t < 0 || t >= len) return;  // the merge kernel writes zeros for such rows
+  const int n_c = (t + 1) / D.B;
+  const int n_sel = min(n_c, D.k);
+  const bool trailing = n_c * D.B <= t;
+  const int n_items = n_sel + (trailing ? 1 : 0);
+  const int item0 = split * kItems;
+  if (item0 >= n_items) return;
+  const int n_mine = min(kItems, n_items - item0);
+  const int32_t *srow = P.sel + (size_t)b * S.n_q * D.k;  // decode: one query row per sequence
+
+  // block start (relative key position) and number of valid keys of item i
+  auto item_block = [&](int i, int &key0, int &nkeys) {
+    if (i < n_sel) {
+      key0 = srow[i] * D.B;
+      nkeys = kBlk;
+    } else {
+      key0 = n_c * D.B;
+      nkeys = t + 1 - key0;
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kItems; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int z = b * D.Hkv + g;
+    for (int i = 0; i < n_mine; ++i) {
+      int key0, nk;
+      item_block(item0 + i, key0, nk);
+      mbar_arrive_expect_tx(&bars[i], 4 * (kTileBytes / 2));
+      uint8_t *kd = ks + i * kTileBytes, *vd = vs + i * kTileBytes;
+      tma_load_3d(&tm_k, &bars[i], kd, 0, start + key0, z);
+      tma_load_3d(&tm_k, &bars[i], kd + kTileBytes / 2, 64, start + key0, z);
+      tma_load_3d(&tm_v, &bars[i], vd, 0, start + key0, z);
+      tma_load_3d(&tm_v, &bars[i], vd + kTileBytes / 2, 64, start + key0, z);
+    }
+  }
+
+  // q of the group as the A operand: rows = heads (0..G-1, rest zero), 8 k-steps of 16 dims.
+  const int head = lane >> 2;  // A/C row owned by this lane (rows 8..15 are padding)
+  const int G = D.G;
+  uint32_t qa[8][2];
+  {
+    const __nv_bfloat16 *qrow = P.q + (((size_t)b * S.n_q) * D.Hq + (size_t)g * G + head) * kD;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int c0 = kk * 16 + 2 * (lane & 3);
+      if (head < G) {
+        qa[kk][0] = *(const uint32_t *)(qrow + c0);
+        qa[kk][1] = *(const uint32_t *)(qrow + c0 + 8);
+      } else {
+        qa[kk][0] = qa[kk][1] = 0u;
+      }
+    }
+  }
+  const float sl2 = D.scale * 1.4426950408889634f;
+  float m = -INFINITY, l = 0.f;
+  float o[16][4];
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+
+  bool fail = false;
+  for (int i = 0; i < n_mine; ++i) {
+    int key0, nk;
+    item_block(item0 + i, key0, nk);
+    if (!mbar_wait(&bars[i], 0, kWaitNs)) {
+      fail = true;
+      break;
+    }
+    const uint32_t kb = smem_u32(ks + i * kTileBytes), vb = smem_u32(vs + i * kTileBytes);
+    if (nk < kBlk) {
+      // zero V rows past the sequence end (generic writes, read below by ldmatrix)
+      uint8_t *vd = vs + i * kTileBytes;
+      for (int e = threadIdx.x; e < (kBlk - nk) * 16; e += kThreads) {
+        const int rr = nk + e / 16, cc = e % 16;
+        *(uint4 *)(vd + (cc >> 3) * (kTileBytes / 2) + rr * 128 + ((cc & 7) << 4)) = make_uint4(0, 0, 0, 0);
+      }
+      __syncthreads();
+    }
+    // this warp's 16 keys of the block: rows 16 warp .. 16 warp + 15
+    const int r0 = warp * 16;
+    float s[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      // B fragments (K^T, col-major) for 2 key tiles: rows = keys, 16-byte chunks of dims.
+      const int half = kk >> 2;
+      const int mtx = lane >> 3, rr = lane & 7;
+      const int key = r0 + (mtx >> 1) * 8 + rr;
+      const int chunk = (kk & 3) * 2 + (mtx & 1);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(kb + half * (kTileBytes / 2) + sw128(key, chunk), b0, b1, b2, b3);
+      mma16816(s[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+      mma16816(s[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
+    }
+    // mask and online softmax for row `head` over this warp's 16 keys
+    float x[4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int key = r0 + nt * 8 + 2 * (lane & 3) + e;
+        x[nt * 2 + e] = key < nk ? s[nt][e] * sl2 : -INFINITY;
+      }
+    float cmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
+    cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
+    const float m_new = fmaxf(m, cmax);
+    const float corr = (m_new == -INFINITY) ? 1.f : ex2_approx(m - m_new);
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] = (x[e] == -INFINITY) ? 0.f : ex2_approx(x[e] - m_new);
+    float ps = (p[0] + p[1]) + (p[2] + p[3]);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+    l = l * corr + ps;
+    m = m_new;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      o[nt][0] *= corr;
+      o[nt][1] *= corr;
+    }
+    // P (rows = heads, 16 keys) as the A operand; rows 8..15 are zero.
+    const uint32_t pa0 = pack_bf16x2(p[0], p[1]);
+    const uint32_t pa2 = pack_bf16x2(p[2], p[3]);
+    // O += P V: B = V (16 keys x 8 dims per tile), loaded transposed from [key][dim] rows.
+#pragma unroll
+    for (int nt2 = 0; nt2 < 8; ++nt2) {
+      const int mtx = lane >> 3, rr = lane & 7;
+      const int key = r0 + (mtx & 1) * 8 + rr;
+      const int dim_chunk = nt2 * 2 + (mtx >> 1);  // 16-byte chunk of 8 dims (0..15)
+      uint32_t v0, v1, v2, v3;
+      ldsm_x4_t(vb + (dim_chunk >> 3) * (kTileBytes / 2) + sw128(key, dim_chunk & 7), v0, v1, v2, v3);
+      mma16816(o[2 * nt2], pa0, 0u, pa2, 0u, v0, v1);
+      mma16816(o[2 * nt2 + 1], pa0, 0u, pa2, 0u, v2, v3);
+    }
+  }
+  if (fail) {
+    record_status(P.status, QSA_ERR_TIMEOUT);
+    return;
+  }
+  // merge the warps: each lane of a quad holds dims 8 nt + 2 (lane & 3) + {0,1} of row `head`
+  float *wm = red;                        // [warps][8]
+  float *wl = red + kWarps * 8;           // [warps][8]
+  float *wo = red + 2 * kWarps * 8;       // [warps][8][128]
+  if ((lane & 3) == 0 && head < kMaxG) {
+    wm[warp * 8 + head] = m;
+    wl[warp * 8 + head] = l;
+  }
+  if (head < kMaxG) {
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      const int dcol = nt * 8 + 2 * (lane & 3);
+      wo[(warp * 8 + head) * kD + dcol] = o[nt][0];
+      wo[(warp * 8 + head) * kD + dcol + 1] = o[nt][1];
+    }
+  }
+  __syncthreads();
+  float *dst = P.part + (((size_t)b * D.Hkv + g) * P.max_splits + split) * G * (kD + 2);
+  for (int e = threadIdx.x; e < G * kD; e += kThreads) {
+    const int hh = e / kD, dd = e % kD;
+    float mm = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, wm[w * 8 + hh]);
+    float acc = 0.f, ll = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      const float f = (wm[w * 8 + hh] == -INFINITY) ? 0.f : ex2_approx(wm[w * 8 + hh] - mm);
+      acc += f * wo[(w * 8 + hh) * kD + dd];
+      ll += f * wl[w * 8 + hh];
+    }
+    dst[hh * (kD + 2) + dd] = acc;
+    if (dd == 0) {
+      dst[hh * (kD + 2) + kD] = mm;
+      dst[hh * (kD + 2) + kD + 1] = ll;
+    }
+  }
+}
+
+// Merge the splits of each (sequence, query head): O = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
+__global__ void __launch_bounds__(kD) k_decode_merge(DecParams P) {
+  const Dims &D = P.D;
+  const Seqs &S = P.S;
+  const int h = blockIdx.x, b = blockIdx.y, dd = threadIdx.x;
+  const int g = h / D.G, hh = h % D.G;
+  __nv_bfloat16 *orow = P.out + ((size_t)b * S.n_q * D.Hq + h) * kD;
+  const bool ok = seq_ok(S, b, nullptr);
+  const int len = ok ? S.kv_len[b] : 0;
+  const int t = seq_qfirst(S, b);
+  if (!ok || t < 0 || t >= len) {
+    orow[dd] = __float2bfloat16_rn(0.f);
+    return;
+  }
+  const int n_c = (t + 1) / D.B;
+  const int n_items = min(n_c, D.k) + ((n_c * D.B <= t) ? 1 : 0);
+  const int n_splits = (n_items + kItems - 1) / kItems;
+  const float *src = P.part + (((size_t)b * D.Hkv + g) * P.max_splits) * D.G * (kD + 2) + hh * (kD + 2);
+  const size_t stride = (size_t)D.G * (kD + 2);
+  float mm = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) mm = fmaxf(mm, src[s * stride + kD]);
+  float acc = 0.f, ll = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const float ms = src[s * stride + kD];
+    const float f = (ms == -INFINITY) ? 0.f : ex2_approx(ms - mm);
+    acc += f * src[s * stride + dd];
+    ll += f * src[s * stride + kD + 1];
+  }
+  orow[dd] = __float2bfloat16_rn(ll > 0.f ? acc / ll : 0.f);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+bool make_kv_map(CUtensorMap *m, const void *ptr, const Dims &D, const Seqs &S) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)S.kv_cap, (cuuint64_t)S.batch * D.Hkv};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)S.kv_cap * kD * 2};
+  cuuint32_t box[3] = {64, kBlk, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int max_splits_for(const Dims &D) { return (D.k + 1 + kItems - 1) / kItems; }
+
+}  // namespace
+
+bool attn_decode_supported(const Dims &D) { return D.bf16 && D.d == kD && D.B == kBlk && D.G <= kMaxG; }
+
+size_t attn_decode_workspace(const Dims &D, const Seqs &S) {
+  return (size_t)S.batch * D.Hkv * max_splits_for(D) * D.G * (kD + 2) * sizeof(float);
+}
+
+cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
+                               const int32_t *sel, void *out, void *scratch, size_t scratch_bytes, int *status,
+                               cudaStream_t st) {
+  if (!attn_decode_supported(D) || S.n_q != 1) return cudaErrorNotSupported;
+  if (S.batch == 0) return cudaSuccess;
+  if (scratch_bytes < attn_decode_workspace(D, S)) return cudaErrorInvalidValue;
+  CUtensorMap tk, tv;
+  if (!make_kv_map(&tk, k, D, S) || !make_kv_map(&tv, v, D, S)) return cudaErrorInvalidValue;
+  DecParams P;
+  P.D = D;
+  P.S = S;
+  P.q = (const __nv_bfloat16 *)q;
+  P.sel = sel;
+  P.out = (__nv_bfloat16 *)out;
+  P.part = (float *)scratch;
+  P.max_splits = max_splits_for(D);
+  P.status = status;
+  const size_t smem = 1024 + 2 * kItems * kTileBytes + 64 + sizeof(float) * (2 * kWarps * 8 + kWarps * 8 * kD);
+  cudaError_t e = ensure_smem(k_attn_decode, smem);
+  if (e != cudaSuccess) return e;
+  note_launch(2);
+  k_attn_decode<<<dim3(P.max_splits, D.Hkv, S.batch), kThreads, smem, st>>>(tk, tv, P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_decode_merge<<<dim3(D.Hq, S.batch), kD, 0, st>>>(P);
+  return cudaGetLastError();
+}
+
 }  // namespace qsa

@@ -61,6 +61,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 // Host-side count of kernel launches issued by this library.
 void note_launch(int n = 1);
 
+// Remember a failed CUDA call for qsa_last_error() (what + the CUDA error text).
+void note_error(const char *what, cudaError_t e);
+
 // Raise a kernel's dynamic shared memory limit once (the attribute is sticky), so
 // that launches stay legal while a stream is being captured into a CUDA graph.
 template <typename K>

@@ -150,6 +150,110 @@ __global__ void k_score_topk_simt(Dims D, Seqs S, const T *__restrict__ qi,
 }
 
 // ---------------------------------------------------------------------------
+// Steps 2+3 with one CTA per query row (few rows, e.g. a decode step): the row's
+// candidates are spread over all threads, and the same exact radix select runs
+// with block-wide counts; selected ids are written in ascending order.
+// ---------------------------------------------------------------------------
+constexpr int kRowThreads = 256;
+
+__device__ __forceinline__ int block_sum(int v, int *red) {
+  v = __reduce_add_sync(kFull, v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int tot = 0;
+#pragma unroll
+  for (int w = 0; w < kRowThreads / 32; ++w) tot += red[w];
+  return tot;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads)
+k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *__restrict__ kbar,
+                 int32_t *__restrict__ sel, int *status) {
+  extern __shared__ float smem[];
+  const int HD = D.Hi * D.di;
+  float *qi_s = smem;                               // [Hi*di]
+  uint32_t *keys = (uint32_t *)(qi_s + HD);         // [nb_cap]
+  __shared__ int red[kRowThreads / 32];
+  __shared__ int wbase[kRowThreads / 32 + 1];
+  const int r = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool ok = seq_ok(S, b, tid == 0 ? status : nullptr);
+  const int len = ok ? S.kv_len[b] : 0;
+  const int t = seq_qfirst(S, b) + r;
+  const bool valid = ok && t >= 0 && t < len;
+  const int n_c = valid ? (t + 1) / D.B : 0;
+  int32_t *out = sel + ((size_t)b * S.n_q + r) * D.k;
+  if (n_c <= D.k) {
+    for (int i = tid; i < D.k; i += kRowThreads) out[i] = (i < n_c) ? i : -1;
+    return;
+  }
+  const T *src = qi + ((size_t)b * S.n_q + r) * HD;
+  for (int i = tid; i < HD; i += kRowThreads) qi_s[i] = to_f(src[i]);
+  __syncthreads();
+  const float *kb = kbar + (size_t)b * S.nb_cap * D.di;
+  for (int j = tid; j < n_c; j += kRowThreads) {
+    const float4 *kr = (const float4 *)(kb + (size_t)j * D.di);
+    float s = 0.f;
+    for (int h = 0; h < D.Hi; ++h) {
+      const float4 *qh = (const float4 *)(qi_s + h * D.di);
+      float dot = 0.f;
+      for (int c = 0; c < D.di / 4; ++c) {
+        const float4 a = qh[c], kv = kr[c];
+        dot = fmaf(a.x, kv.x, dot);
+        dot = fmaf(a.y, kv.y, dot);
+        dot = fmaf(a.z, kv.z, dot);
+        dot = fmaf(a.w, kv.w, dot);
+      }
+      s += dot > 0.f ? dot : 0.f;
+    }
+    keys[j] = __float_as_uint(s);
+  }
+  __syncthreads();
+  uint32_t prefix = 0;
+  int remaining = D.k;
+  for (int bit = 30; bit >= 0; --bit) {
+    const uint32_t want = (prefix >> bit) | 1u;
+    int cnt = 0;
+    for (int j = tid; j < n_c; j += kRowThreads) cnt += ((keys[j] >> bit) == want);
+    cnt = block_sum(cnt, red);
+    if (cnt >= remaining) prefix |= (1u << bit);
+    else remaining -= cnt;
+  }
+  // ascending compaction: chunks of kRowThreads consecutive ids in thread order
+  const unsigned lt = lanemask_lt();
+  int base = 0, tie_base = 0;
+  for (int j0 = 0; j0 < n_c; j0 += kRowThreads) {
+    const int j = j0 + tid;
+    const uint32_t key = j < n_c ? keys[j] : 0u;
+    const bool gt = j < n_c && key > prefix;
+    const bool eq = j < n_c && key == prefix;
+    // ranks of the ties in id order decide which ties are kept
+    const unsigned eq_mask = __ballot_sync(kFull, eq);
+    __syncthreads();
+    if (lane == 0) red[warp] = __popc(eq_mask);
+    __syncthreads();
+    int eq_before = tie_base;
+    for (int w = 0; w < warp; ++w) eq_before += red[w];
+    int eq_tot = 0;
+    for (int w = 0; w < kRowThreads / 32; ++w) eq_tot += red[w];
+    const bool take = gt || (eq && eq_before + __popc(eq_mask & lt) < remaining);
+    const unsigned take_mask = __ballot_sync(kFull, take);
+    if (lane == 0) wbase[warp] = __popc(take_mask);
+    __syncthreads();
+    int take_before = base;
+    for (int w = 0; w < warp; ++w) take_before += wbase[w];
+    int take_tot = 0;
+    for (int w = 0; w < kRowThreads / 32; ++w) take_tot += wbase[w];
+    if (take) out[take_before + __popc(take_mask & lt)] = j;
+    base += take_tot;
+    tie_base += eq_tot;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Step 4 on CUDA cores. One CTA per (query row, KV head, sequence); one warp per
 // query head of the group. Keys stream in chunks of 32 through shared memory
 // (selected blocks in ascending order, then the trailing range); each warp keeps
@@ -309,6 +413,25 @@ static size_t score_smem(const Dims &D, int warps, int nc_cap) {
 cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
                                    int32_t *sel, int *status, cudaStream_t st) {
   if (S.batch == 0 || S.n_q == 0) return cudaSuccess;
+  if ((long long)S.batch * S.n_q <= 4096 && D.di % 4 == 0) {
+    // few rows: one CTA per row
+    const size_t smem = sizeof(float) * ((size_t)D.Hi * D.di + S.nb_cap);
+    if (smem <= 200 * 1024) {
+      dim3 grid(S.n_q, S.batch);
+      note_launch();
+      cudaError_t e;
+      if (D.bf16) {
+        auto kern = k_score_topk_row<__nv_bfloat16>;
+        if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
+        kern<<<grid, kRowThreads, smem, st>>>(D, S, (const __nv_bfloat16 *)qi, kbar, sel, status);
+      } else {
+        auto kern = k_score_topk_row<float>;
+        if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
+        kern<<<grid, kRowThreads, smem, st>>>(D, S, (const float *)qi, kbar, sel, status);
+      }
+      return cudaGetLastError();
+    }
+  }
   const int nc_cap = S.nb_cap;
   int warps = S.n_q < 8 ? S.n_q : 8;
   const size_t limit = 200 * 1024;

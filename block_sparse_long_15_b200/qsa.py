@@ -25,7 +25,8 @@ QSA_PREFILL, QSA_DECODE = 0, 1
 class QSAError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        detail = f" [{qsa_last_error()}]" if status == QSA_ERR_CUDA else ""
+        super().__init__(f"{where}: {status_string(status)} (status {status}){detail}")
 
 
 class qsa_config_t(ctypes.Structure):
@@ -66,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "qsa_abi_version": ([], I),
         "qsa_attn_kernel_name": ([cfgp, I], ctypes.c_char_p),
         "qsa_kernel_launch_count": ([], ctypes.c_uint64),
+        "qsa_last_error": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -78,7 +80,7 @@ _lib = _load()
 EXPORTED = ("qsa_config_validate", "qsa_topk_blocks", "qsa_status_string", "qsa_workspace_size",
             "qsa_compress_blocks", "qsa_index_score_topk", "qsa_sparse_attn", "qsa_forward",
             "qsa_read_device_status", "qsa_abi_version", "qsa_attn_kernel_name",
-            "qsa_kernel_launch_count")
+            "qsa_kernel_launch_count", "qsa_last_error")
 
 
 def library() -> ctypes.CDLL:
@@ -149,6 +151,10 @@ def qsa_abi_version() -> int:
 
 def qsa_attn_kernel_name(cfg: qsa_config_t, mode: int = QSA_PREFILL) -> str:
     return _lib.qsa_attn_kernel_name(ctypes.byref(cfg), mode).decode()
+
+
+def qsa_last_error() -> str:
+    return _lib.qsa_last_error().decode()
 
 
 def qsa_kernel_launch_count() -> int:

@@ -187,6 +187,9 @@ const char *qsa_attn_kernel_name(const qsa_config_t *cfg, int32_t mode);
  * counter bumped at every launch; diagnostics and benchmarking). */
 uint64_t qsa_kernel_launch_count(void);
 
+/* Text of the last CUDA error this library saw on the calling thread ("" if none). */
+const char *qsa_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif
