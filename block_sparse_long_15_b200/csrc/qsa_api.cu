@@ -133,6 +133,8 @@ qsa_status_t attn_dispatch(const Dims &D, const Seqs &S, const void *q, const vo
 
 }  // namespace
 
+qsa_status_t qsa::resolve_config(const qsa_config_t *cfg, Dims *D) { return resolve(cfg, D); }
+
 extern "C" {
 
 int32_t qsa_abi_version(void) { return QSA_ABI_VERSION; }

@@ -18,6 +18,8 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "qsa_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -367,3 +369,92 @@ cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, cons
 }
 
 }  // namespace qsa
+
+// ---------------------------------------------------------------------------
+// Decode attention without a caller workspace.
+//
+// Some callers cannot hand this library any device memory beyond their inputs
+// and outputs: for example a plugin that a host framework invokes with only its
+// input and output buffers, or a serving process whose device memory is all
+// reserved up front by its own pool, so that a cudaMalloc would fail or bypass
+// that pool. For them this entry point keeps the split partials of the decode
+// kernel in a fixed array in the library's device memory instead of a workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Split partials of qsa_sparse_attn_decode_noalloc: every GPU that loads the
+// library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QSA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[256];  // device address of the array, per device ordinal
+
+// Device address of the array on the current device. The array's name is only a
+// host-side stand-in in host code; its device address comes from
+// cudaGetSymbolAddress, called once per device with that device current.
+cudaError_t noalloc_scratch(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" qsa_status_t qsa_sparse_attn_decode_noalloc(const qsa_config_t *cfg, const void *q, const void *k,
+                                                       const void *v, const int32_t *sel,
+                                                       const int32_t *kv_start, const int32_t *kv_len,
+                                                       int32_t batch, int32_t kv_cap, void *out,
+                                                       qsa_stream_t stream) {
+  using namespace qsa;
+  Dims D;
+  qsa_status_t s = resolve_config(cfg, &D);
+  if (s != QSA_OK) return s;
+  if (batch < 0 || kv_cap < 0) return QSA_ERR_INVALID_ARG;
+  if (batch == 0) return QSA_OK;
+  if (!q || !k || !v || !sel || !kv_start || !kv_len || !out) return QSA_ERR_INVALID_ARG;
+  const void *ptrs[] = {q, k, v, sel, out};
+  for (const void *p : ptrs)
+    if (((uintptr_t)p & 15u) != 0) return QSA_ERR_INVALID_ARG;
+  if (!attn_decode_supported(D)) return QSA_ERR_UNSUPPORTED;
+  Seqs S;
+  S.kv_start = kv_start;
+  S.kv_len = kv_len;
+  S.q_first = nullptr;  // the query of sequence b sits at kv_len[b] - 1
+  S.batch = batch;
+  S.n_q = 1;
+  S.kv_cap = kv_cap;
+  S.nb_cap = kv_cap / D.B;
+  const size_t need = attn_decode_workspace(D, S);
+  if (need > (size_t)QSA_NOALLOC_SCRATCH_BYTES) {
+    char what[160];
+    snprintf(what, sizeof what, "decode partials need %zu bytes, more than the %d-byte static scratch", need,
+             (int)QSA_NOALLOC_SCRATCH_BYTES);
+    note_error(what, cudaErrorInvalidValue);
+    return QSA_ERR_UNSUPPORTED;
+  }
+  void *scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) {
+    note_error("cudaGetSymbolAddress of the static decode scratch", e);
+    return QSA_ERR_CUDA;
+  }
+  // No device-side status word here (it would need a caller buffer or a sync to
+  // read): lengths that do not fit the cache are skipped without a report.
+  e = launch_attn_decode(D, S, q, k, v, sel, out, scratch, need, nullptr, (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    note_error("qsa_sparse_attn_decode_noalloc launch", e);
+    return e == cudaErrorNotSupported ? QSA_ERR_UNSUPPORTED : QSA_ERR_CUDA;
+  }
+  return QSA_OK;
+}
+

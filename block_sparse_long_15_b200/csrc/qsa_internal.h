@@ -58,6 +58,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
   return __float2bfloat16_rn(x);
 }
 
+// Validates a config and fills the resolved shape (the rules of qsa_config_validate).
+qsa_status_t resolve_config(const qsa_config_t *cfg, Dims *D);
+
 // Host-side count of kernel launches issued by this library.
 void note_launch(int n = 1);
 

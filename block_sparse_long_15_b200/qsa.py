@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "qsa_attn_kernel_name": ([cfgp, I], ctypes.c_char_p),
         "qsa_kernel_launch_count": ([], ctypes.c_uint64),
         "qsa_last_error": ([], ctypes.c_char_p),
+        "qsa_sparse_attn_decode_noalloc": ([cfgp, V, V, V, V, V, V, I, I, V, V], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -80,7 +81,10 @@ _lib = _load()
 EXPORTED = ("qsa_config_validate", "qsa_topk_blocks", "qsa_status_string", "qsa_workspace_size",
             "qsa_compress_blocks", "qsa_index_score_topk", "qsa_sparse_attn", "qsa_forward",
             "qsa_read_device_status", "qsa_abi_version", "qsa_attn_kernel_name",
-            "qsa_kernel_launch_count", "qsa_last_error")
+            "qsa_kernel_launch_count", "qsa_last_error", "qsa_sparse_attn_decode_noalloc")
+
+# Size of the library's fixed decode scratch (QSA_NOALLOC_SCRATCH_BYTES in qsa.h).
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 def library() -> ctypes.CDLL:
@@ -222,6 +226,21 @@ def qsa_forward(cfg, mode: int, t: Dict[str, torch.Tensor], workspace, stream=No
                       _p(t["out"]))
     _check(_lib.qsa_forward(ctypes.byref(cfg), mode, ctypes.byref(T), _p(workspace), workspace.numel(),
                             _stream(stream)), "qsa_forward")
+
+
+def qsa_sparse_attn_decode_noalloc(cfg, q, k, v, sel, kv_start, kv_len, out, stream=None):
+    """Decode attention with no workspace: for callers that cannot allocate device
+    memory of their own (a plugin given only its inputs and outputs, a server whose
+    memory is all in its own pool). The partials live in a fixed array inside the
+    library; calls that overlap on the GPU race on it."""
+    batch = q.shape[0]
+    kv_cap = k.shape[2]
+    dt = _elem(cfg)
+    _want(q, dt, (batch, 1, cfg.num_attention_heads, cfg.head_dim), "q")
+    _want(out, dt, (batch, 1, cfg.num_attention_heads, cfg.head_dim), "out")
+    _check(_lib.qsa_sparse_attn_decode_noalloc(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(kv_start),
+                                               _p(kv_len), batch, kv_cap, _p(out), _stream(stream)),
+           "qsa_sparse_attn_decode_noalloc")
 
 
 def qsa_read_device_status(workspace: torch.Tensor, stream=None) -> int:

@@ -190,6 +190,35 @@ uint64_t qsa_kernel_launch_count(void);
 /* Text of the last CUDA error this library saw on the calling thread ("" if none). */
 const char *qsa_last_error(void);
 
+/* Size of the fixed device array that qsa_sparse_attn_decode_noalloc uses. */
+#define QSA_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+
+/* Decode attention (step 4 for one query row per sequence, at kv_len[b] - 1) for
+ * callers that cannot hand the library any device memory besides their inputs and
+ * outputs -- for example a plugin that its host framework calls with nothing but
+ * input and output buffers, or a serving process that reserves all device memory
+ * for its own pool, so that a cudaMalloc would fail or go around that pool. It
+ * computes what qsa_sparse_attn computes for n_q == 1 with q_first[b] = kv_len[b] - 1,
+ * and allocates nothing: the split partials of the decode kernel live in a fixed
+ * array of QSA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits (the paper has no counterpart; this is
+ * an interface convenience).
+ *   Arguments and layouts as for qsa_sparse_attn with n_q = 1 (q, out [batch][1][Hq][d];
+ *   k, v [batch][Hkv][kv_cap][d]; sel [batch][1][k]); bf16, head_dim 128, B = 64, G <= 8.
+ *   The first call on a device looks up the array's device address (with that device
+ *   current); make that first call before any stream capture.
+ *   Every call on a device shares the one array and leaves its partials there; calls
+ *   that overlap on the GPU (e.g. on two streams) race on it and must be serialised
+ *   by the caller.
+ *   Returns QSA_ERR_UNSUPPORTED (and sets qsa_last_error) when the partials of this
+ *   batch, batch * Hkv * ceil((k + 1) / 2) * G * (d + 2) * 4 bytes, exceed the array,
+ *   and for shapes the decode kernel does not serve. No device-side status is kept:
+ *   lengths that do not fit the cache are skipped without a report. */
+qsa_status_t qsa_sparse_attn_decode_noalloc(const qsa_config_t *cfg, const void *q, const void *k,
+                                            const void *v, const int32_t *sel, const int32_t *kv_start,
+                                            const int32_t *kv_len, int32_t batch, int32_t kv_cap, void *out,
+                                            qsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

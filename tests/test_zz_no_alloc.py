@@ -1,0 +1,64 @@
+"""Decode attention without a caller workspace (qsa_sparse_attn_decode_noalloc).
+
+Callers such as a plugin that its host framework gives only input and output
+buffers, or a server whose device memory all sits in its own pool, cannot hand the
+library scratch memory; this entry point keeps the decode partials in a fixed array
+inside the library instead. The GPU test checks it against qsa_sparse_attn with a
+workspace, through the C ABI, on two calls in a row. This file is collected last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from block_sparse_long_15_b200 import workloads as W
+
+ATOL, RTOL = 1e-2, 2e-2  # the bf16 output tolerance of the parity tests
+
+
+def test_sizes_beyond_the_static_scratch_are_rejected_on_host():
+    from block_sparse_long_15_b200 import build
+    build.build()
+    from block_sparse_long_15_b200 import qsa
+    cfg = qsa.make_config(Hq=16, Hkv=2, d=128, Hi=4, di=64, block=64, topk=32)
+    fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check comes first
+    # 512 sequences x 2 KV heads x 17 splits x 8 heads x 130 floats is about 72 MB
+    st = qsa.library().qsa_sparse_attn_decode_noalloc(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake,
+                                                      512, 4096, fake, None)
+    assert st == qsa.QSA_ERR_UNSUPPORTED
+    assert "static scratch" in qsa.qsa_last_error()
+
+
+@pytest.mark.gpu
+def test_noalloc_decode_matches_workspace_path_twice(cuda_lib):
+    qsa = cuda_lib
+    from block_sparse_long_15_b200.runner import QSADecode
+    w = W.small_variant(W.WORKLOADS["bf16_decode_b64_l4k_32k"], seq=8192, batch=24, len_min=700,
+                        len_max=8000)
+    d = QSADecode(w, W.make_inputs(w))
+    d()  # appends the new token and selects the blocks (sel) for this step
+    torch.cuda.synchronize()
+    assert d.status() == qsa.QSA_OK
+    t = d.t
+    q_first = (t["kv_len"] - 1).contiguous()
+    ref = torch.empty_like(t["q"])
+    qsa.qsa_sparse_attn(d.cfg, t["q"], t["k_cache"], t["v_cache"], t["sel"], t["kv_start"], t["kv_len"],
+                        q_first, ref, d.ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(ref.float()).all()
+
+    # first call: the whole batch
+    out1 = torch.full_like(t["q"], float("nan"))
+    qsa.qsa_sparse_attn_decode_noalloc(d.cfg, t["q"], t["k_cache"], t["v_cache"], t["sel"], t["kv_start"],
+                                       t["kv_len"], out1)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out1.float(), ref.float(), atol=ATOL, rtol=RTOL)
+
+    # second call right after: a smaller batch, so the array holds the first call's partials
+    n = 9
+    out2 = torch.full_like(t["q"][:n], float("nan"))
+    qsa.qsa_sparse_attn_decode_noalloc(d.cfg, t["q"][:n].contiguous(), t["k_cache"][:n].contiguous(),
+                                       t["v_cache"][:n].contiguous(), t["sel"][:n].contiguous(),
+                                       t["kv_start"][:n].contiguous(), t["kv_len"][:n].contiguous(), out2)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out2.float(), ref[:n].float(), atol=ATOL, rtol=RTOL)
