@@ -272,14 +272,14 @@ qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensor
   if (mode == QSA_PREFILL) {
     s = cuda_status(launch_compress(D, S, t->ki_cache, nullptr, t->kbar_cache, t->kbar_blocks,
                                     status, st));
+    if (s != QSA_OK) return s;
+    s = cuda_status(launch_score_topk_simt(D, S, t->qi, t->kbar_cache, t->sel, status, st));
   } else {
-    s = cuda_status(launch_decode_append(D, S, t->k_cache, t->v_cache, t->ki_cache, t->kbar_cache,
-                                         t->kbar_blocks, t->k_new, t->v_new, t->ki_new, status, st));
     // The decode query sits at kv_len - 1; a null q_first tells the kernels so.
     S.q_first = nullptr;
+    DecodeAppend A{t->k_cache, t->v_cache, t->ki_cache, t->kbar_blocks, t->k_new, t->v_new, t->ki_new};
+    s = cuda_status(launch_decode_append_score(D, S, A, t->qi, t->kbar_cache, t->sel, status, st));
   }
-  if (s != QSA_OK) return s;
-  s = cuda_status(launch_score_topk_simt(D, S, t->qi, t->kbar_cache, t->sel, status, st));
   if (s != QSA_OK) return s;
   return attn_dispatch(D, S, t->q, t->k_cache, t->v_cache, t->sel, t->out, workspace, workspace_bytes, st);
 }

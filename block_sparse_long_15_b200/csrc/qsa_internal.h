@@ -89,6 +89,17 @@ cudaError_t launch_compress(const Dims &D, const Seqs &S, const void *ki, const 
 cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
                                    int32_t *sel, int *status, cudaStream_t st);
 
+// The decode prologue (append the new token at kv_len - 1, compress a block it
+// completes, advance kbar_blocks; see launch_decode_append) fused with steps 2+3
+// for the single query row of each sequence.
+struct DecodeAppend {
+  void *k_cache, *v_cache, *ki_cache;
+  int32_t *kbar_blocks;
+  const void *k_new, *v_new, *ki_new;
+};
+cudaError_t launch_decode_append_score(const Dims &D, const Seqs &S, const DecodeAppend &A, const void *qi,
+                                       float *kbar, int32_t *sel, int *status, cudaStream_t st);
+
 // Step 4 on CUDA cores (fp32 accumulate), any supported shape.
 cudaError_t launch_attn_simt(const Dims &D, const Seqs &S, const void *q, const void *k,
                              const void *v, const int32_t *sel, void *out, int *status,

@@ -155,6 +155,7 @@ __global__ void k_score_topk_simt(Dims D, Seqs S, const T *__restrict__ qi,
 // with block-wide counts; selected ids are written in ascending order.
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 256;
+constexpr int kMaxHi = 8;  // indexer heads scored together per k̄ piece
 
 __device__ __forceinline__ int block_sum(int v, int *red) {
   v = __reduce_add_sync(kFull, v);
@@ -168,11 +169,59 @@ __device__ __forceinline__ int block_sum(int v, int *red) {
   return tot;
 }
 
+// Decode prologue for sequence b, run by one CTA: check the indexer state is in
+// step (kbar_blocks == (L-1)/B; larger means the cache was cropped, which QSA does
+// not support), append the new token at L-1, and if that completes block
+// j = L/B - 1, compress it and advance kbar_blocks. Ends with a block barrier.
 template <typename T>
+__device__ void decode_append_block(const Dims &D, const Seqs &S, const DecodeAppend &A, float *kbar, int b,
+                                    int *status) {
+  T *k_cache = (T *)A.k_cache, *v_cache = (T *)A.v_cache, *ki_cache = (T *)A.ki_cache;
+  const T *k_new = (const T *)A.k_new, *v_new = (const T *)A.v_new, *ki_new = (const T *)A.ki_new;
+  __shared__ int s_go;
+  if (threadIdx.x == 0) {
+    s_go = 0;
+    if (seq_ok(S, b, status)) {
+      const int L = S.kv_len[b];
+      const int have = A.kbar_blocks[b], need = (L - 1) / D.B;
+      if (L < 1) record_status(status, QSA_ERR_DEVICE_CHECK);
+      else if (have != need) record_status(status, have > need ? QSA_ERR_UNSUPPORTED : QSA_ERR_DEVICE_CHECK);
+      else s_go = 1;
+    }
+  }
+  __syncthreads();
+  if (s_go) {
+    const int L = S.kv_len[b], start = seq_start(S, b);
+    const size_t pos = (size_t)start + L - 1;
+    for (int i = threadIdx.x; i < D.Hkv * D.d; i += blockDim.x) {
+      const int g = i / D.d, c = i - g * D.d;
+      const size_t dst = (((size_t)b * D.Hkv + g) * S.kv_cap + pos) * D.d + c;
+      k_cache[dst] = k_new[(size_t)b * D.Hkv * D.d + i];
+      v_cache[dst] = v_new[(size_t)b * D.Hkv * D.d + i];
+    }
+    for (int c = threadIdx.x; c < D.di; c += blockDim.x)
+      ki_cache[((size_t)b * S.kv_cap + pos) * D.di + c] = ki_new[(size_t)b * D.di + c];
+    if (L % D.B == 0) {
+      __syncthreads();
+      const int j = L / D.B - 1;
+      const T *src = ki_cache + ((size_t)b * S.kv_cap + start + (size_t)j * D.B) * D.di;
+      for (int c = threadIdx.x; c < D.di; c += blockDim.x) {
+        float acc = 0.f;
+        for (int u = 0; u < D.B; ++u) acc += to_f(src[(size_t)u * D.di + c]);
+        kbar[((size_t)b * S.nb_cap + j) * D.di + c] = acc / (float)D.B;
+      }
+      if (threadIdx.x == 0) A.kbar_blocks[b] = L / D.B;
+    }
+  }
+  __syncthreads();
+}
+
+template <typename T, bool kAppend>
 __global__ void __launch_bounds__(kRowThreads)
-k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *__restrict__ kbar,
-                 int32_t *__restrict__ sel, int *status) {
+k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, int32_t *__restrict__ sel,
+                 int *status, DecodeAppend A) {
   extern __shared__ float smem[];
+  if (kAppend) decode_append_block<T>(D, S, A, (float *)kbar, blockIdx.y, status);
   const int HD = D.Hi * D.di;
   float *qi_s = smem;                               // [Hi*di]
   uint32_t *keys = (uint32_t *)(qi_s + HD);         // [nb_cap]
@@ -195,32 +244,88 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *__restri
   __syncthreads();
   const float *kb = kbar + (size_t)b * S.nb_cap * D.di;
   for (int j = tid; j < n_c; j += kRowThreads) {
+    // the candidate's k̄ row is read in 64-float pieces whose 16 loads are all in
+    // flight together; the query heads (up to kMaxHi at a time) reuse each piece
     const float4 *kr = (const float4 *)(kb + (size_t)j * D.di);
     float s = 0.f;
-    for (int h = 0; h < D.Hi; ++h) {
-      const float4 *qh = (const float4 *)(qi_s + h * D.di);
-      float dot = 0.f;
-      for (int c = 0; c < D.di / 4; ++c) {
-        const float4 a = qh[c], kv = kr[c];
-        dot = fmaf(a.x, kv.x, dot);
-        dot = fmaf(a.y, kv.y, dot);
-        dot = fmaf(a.z, kv.z, dot);
-        dot = fmaf(a.w, kv.w, dot);
+    for (int h0 = 0; h0 < D.Hi; h0 += kMaxHi) {
+      float dot[kMaxHi];
+#pragma unroll
+      for (int h = 0; h < kMaxHi; ++h) dot[h] = 0.f;
+      for (int c0 = 0; c0 < D.di / 4; c0 += 16) {
+        float4 kv[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) kv[c] = (c0 + c < D.di / 4) ? __ldg(&kr[c0 + c]) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < kMaxHi; ++h) {
+          if (h0 + h >= D.Hi) break;
+          const float4 *qh = (const float4 *)(qi_s + (h0 + h) * D.di) + c0;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            if (c0 + c >= D.di / 4) break;
+            const float4 a = qh[c];
+            dot[h] = fmaf(a.x, kv[c].x, dot[h]);
+            dot[h] = fmaf(a.y, kv[c].y, dot[h]);
+            dot[h] = fmaf(a.z, kv[c].z, dot[h]);
+            dot[h] = fmaf(a.w, kv[c].w, dot[h]);
+          }
+        }
       }
-      s += dot > 0.f ? dot : 0.f;
+#pragma unroll
+      for (int h = 0; h < kMaxHi; ++h)
+        if (h0 + h < D.Hi) s += dot[h] > 0.f ? dot[h] : 0.f;
     }
     keys[j] = __float_as_uint(s);
   }
   __syncthreads();
-  uint32_t prefix = 0;
+  // Radix select of the k-th largest key, 8 bits at a time from the top: count the
+  // keys that match the prefix found so far per value of the next byte, then keep
+  // the byte at which the running count from the top reaches `remaining`.
+  __shared__ int hist[256];
+  __shared__ int s_digit, s_above;
+  uint32_t prefix = 0, pmask = 0;
   int remaining = D.k;
-  for (int bit = 30; bit >= 0; --bit) {
-    const uint32_t want = (prefix >> bit) | 1u;
-    int cnt = 0;
-    for (int j = tid; j < n_c; j += kRowThreads) cnt += ((keys[j] >> bit) == want);
-    cnt = block_sum(cnt, red);
-    if (cnt >= remaining) prefix |= (1u << bit);
-    else remaining -= cnt;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kRowThreads) hist[i] = 0;
+    __syncthreads();
+    for (int j = tid; j < n_c; j += kRowThreads) {
+      const uint32_t key = keys[j];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane L owns bytes 255-8L .. 248-8L (descending)
+      int c[8], tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        c[q] = hist[255 - 8 * lane - q];
+        tot += c[q];
+      }
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - tot;  // keys in higher bytes than this lane's range
+      if (excl < remaining && incl >= remaining) {
+        int above = excl;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (above + c[q] >= remaining) {
+            s_digit = 255 - 8 * lane - q;
+            s_above = above;
+            break;
+          }
+          above += c[q];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= (uint32_t)s_digit << shift;
+    pmask |= 255u << shift;
+    remaining -= s_above;
+    __syncthreads();
   }
   // ascending compaction: chunks of kRowThreads consecutive ids in thread order
   const unsigned lt = lanemask_lt();
@@ -421,13 +526,13 @@ cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi,
       note_launch();
       cudaError_t e;
       if (D.bf16) {
-        auto kern = k_score_topk_row<__nv_bfloat16>;
+        auto kern = k_score_topk_row<__nv_bfloat16, false>;
         if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
-        kern<<<grid, kRowThreads, smem, st>>>(D, S, (const __nv_bfloat16 *)qi, kbar, sel, status);
+        kern<<<grid, kRowThreads, smem, st>>>(D, S, (const __nv_bfloat16 *)qi, kbar, sel, status, DecodeAppend{});
       } else {
-        auto kern = k_score_topk_row<float>;
+        auto kern = k_score_topk_row<float, false>;
         if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
-        kern<<<grid, kRowThreads, smem, st>>>(D, S, (const float *)qi, kbar, sel, status);
+        kern<<<grid, kRowThreads, smem, st>>>(D, S, (const float *)qi, kbar, sel, status, DecodeAppend{});
       }
       return cudaGetLastError();
     }
@@ -451,6 +556,32 @@ cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi,
     e = ensure_smem(kern, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, warps * 32, smem, st>>>(D, S, (const float *)qi, kbar, sel, status, warps, nc_cap);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_append_score(const Dims &D, const Seqs &S, const DecodeAppend &A, const void *qi,
+                                       float *kbar, int32_t *sel, int *status, cudaStream_t st) {
+  if (S.batch == 0) return cudaSuccess;
+  const size_t smem = sizeof(float) * ((size_t)D.Hi * D.di + S.nb_cap);
+  if (S.n_q != 1 || D.di % 4 != 0 || smem > 200 * 1024) {
+    // general path: separate prologue, then the scoring launch
+    cudaError_t e = launch_decode_append(D, S, A.k_cache, A.v_cache, A.ki_cache, kbar, A.kbar_blocks, A.k_new,
+                                         A.v_new, A.ki_new, status, st);
+    if (e != cudaSuccess) return e;
+    return launch_score_topk_simt(D, S, qi, kbar, sel, status, st);
+  }
+  dim3 grid(1, S.batch);
+  note_launch();
+  cudaError_t e;
+  if (D.bf16) {
+    auto kern = k_score_topk_row<__nv_bfloat16, true>;
+    if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
+    kern<<<grid, kRowThreads, smem, st>>>(D, S, (const __nv_bfloat16 *)qi, kbar, sel, status, A);
+  } else {
+    auto kern = k_score_topk_row<float, true>;
+    if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
+    kern<<<grid, kRowThreads, smem, st>>>(D, S, (const float *)qi, kbar, sel, status, A);
   }
   return cudaGetLastError();
 }

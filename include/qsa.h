@@ -126,10 +126,11 @@ int32_t qsa_topk_blocks(const qsa_config_t *cfg);
 const char *qsa_status_string(qsa_status_t status);
 
 /* Bytes of workspace the calls below need for these sizes (mode QSA_PREFILL or
- * QSA_DECODE). The workspace is caller-owned device memory, 256-byte aligned; its
- * first 256 bytes hold the status word, which must be zero before first use
- * (qsa_read_device_status clears it). One workspace must not serve two calls
- * that run concurrently. */
+ * QSA_DECODE). The workspace is caller-owned device memory, 256-byte aligned, and
+ * must be all zero before its first use; the library leaves the parts it relies on
+ * at zero again after each call. Its first 256 bytes hold the status word
+ * (qsa_read_device_status reads and clears it). One workspace must not serve two
+ * calls that run concurrently. */
 qsa_status_t qsa_workspace_size(const qsa_config_t *cfg, int32_t mode, int32_t batch, int32_t n_q,
                                 int32_t kv_cap, size_t *bytes);
 
@@ -211,8 +212,9 @@ const char *qsa_last_error(void);
  *   that overlap on the GPU (e.g. on two streams) race on it and must be serialised
  *   by the caller.
  *   Returns QSA_ERR_UNSUPPORTED (and sets qsa_last_error) when the partials of this
- *   batch, batch * Hkv * ceil((k + 1) / 2) * G * (d + 2) * 4 bytes, exceed the array,
- *   and for shapes the decode kernel does not serve. No device-side status is kept:
+ *   batch exceed the array -- with batch * Hkv <= 2048 they take about
+ *   (batch * Hkv + 1024) * G * (d + 2) * 4 bytes, which fits up to that limit for
+ *   G = 8, d = 128 -- and for shapes the decode kernel does not serve. No device-side status is kept:
  *   lengths that do not fit the cache are skipped without a report. */
 qsa_status_t qsa_sparse_attn_decode_noalloc(const qsa_config_t *cfg, const void *q, const void *k,
                                             const void *v, const int32_t *sel, const int32_t *kv_start,

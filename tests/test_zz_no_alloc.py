@@ -22,9 +22,11 @@ def test_sizes_beyond_the_static_scratch_are_rejected_on_host():
     from block_sparse_long_15_b200 import qsa
     cfg = qsa.make_config(Hq=16, Hkv=2, d=128, Hi=4, di=64, block=64, topk=32)
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check comes first
-    # 512 sequences x 2 KV heads x 17 splits x 8 heads x 130 floats is about 72 MB
+    # 2000 sequences x 2 KV heads: past the streaming kernel's unit limit, and the
+    # per-split partials (17 splits x 8 heads x 130 floats per unit, about 283 MB)
+    # do not fit the 16 MiB array
     st = qsa.library().qsa_sparse_attn_decode_noalloc(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake,
-                                                      512, 4096, fake, None)
+                                                      2000, 4096, fake, None)
     assert st == qsa.QSA_ERR_UNSUPPORTED
     assert "static scratch" in qsa.qsa_last_error()
 
