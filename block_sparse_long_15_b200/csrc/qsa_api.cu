@@ -7,6 +7,7 @@
 #include "qsa_internal.h"
 
 #include <atomic>
+#include <mutex>
 
 using namespace qsa;
 
@@ -17,6 +18,31 @@ static std::atomic<uint64_t> g_launches{0};
 static thread_local char g_last_error[256] = "";
 static thread_local uint64_t g_error_serial = 0;
 void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+cudaError_t ensure_smem_for(const void *kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  struct Grant {
+    const void *kernel;
+    int dev;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static Grant table[256];
+  static int n = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  Grant *g = nullptr;
+  for (int i = 0; i < n; ++i)
+    if (table[i].kernel == kernel && table[i].dev == dev) g = &table[i];
+  if (g && g->bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  if (!g && n < 256) g = &table[n++];
+  if (g) *g = Grant{kernel, dev, bytes};
+  return cudaSuccess;
+}
+
 void note_error(const char *what, cudaError_t e) {
   snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
   ++g_error_serial;
@@ -92,6 +118,14 @@ AttnKernel pick_attn(const Dims &D, const Seqs &S) {
   return kAttnSimt;
 }
 
+// Scoring: few rows (a decode step) take the CTA-per-row kernel; otherwise the
+// tensor-core kernel when it serves the shape, else the warp-per-row kernel.
+bool use_score_tc(const Dims &D, const Seqs &S) {
+  return (long long)S.batch * S.n_q > 4096 && score_tc_supported(D, S);
+}
+
+// Scratch after the status word. Scoring and attention run one after the other on
+// the stream, so they share it.
 size_t scratch_need(const Dims &D, const Seqs &S) {
   size_t s = 0;
   switch (pick_attn(D, S)) {
@@ -99,8 +133,10 @@ size_t scratch_need(const Dims &D, const Seqs &S) {
     case kAttnTc: s = attn_tc_workspace(D, S); break;
     default: break;
   }
+  if (use_score_tc(D, S)) s = s > score_tc_workspace(D, S) ? s : score_tc_workspace(D, S);
   return (s + 255) & ~(size_t)255;
 }
+
 
 // Status of a launch; the launch sites record a detailed message, this records a
 // generic one only when no message was recorded since the call began.
@@ -116,6 +152,14 @@ qsa_status_t cuda_status(cudaError_t e) {
 }
 
 int *status_word(void *ws) { return (int *)ws; }
+
+qsa_status_t score_dispatch(const Dims &D, const Seqs &S, const void *qi, const float *kbar, int32_t *sel,
+                            void *ws, cudaStream_t st) {
+  int *status = (int *)ws;
+  if (use_score_tc(D, S))
+    return cuda_status(launch_score_topk_tc(D, S, qi, kbar, sel, (char *)ws + kStatusBytes, status, st));
+  return cuda_status(launch_score_topk_simt(D, S, qi, kbar, sel, status, st));
+}
 
 qsa_status_t attn_dispatch(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
                            const int32_t *sel, void *out, void *ws, size_t ws_bytes, cudaStream_t st) {
@@ -216,11 +260,11 @@ qsa_status_t qsa_index_score_topk(const qsa_config_t *cfg, const void *qi, const
     return QSA_ERR_INVALID_ARG;
   if (!aligned16(qi) || !aligned16(kbar) || !aligned16(sel) || !aligned16(workspace))
     return QSA_ERR_INVALID_ARG;
-  if (workspace_bytes < kStatusBytes) return QSA_ERR_INVALID_ARG;
   // Scoring reads no keys, only k̄ rows (indexed by block from the sequence start),
   // so kv_start is not needed here.
   Seqs S = make_seqs(D, nullptr, kv_len, q_first, batch, n_q, kv_cap);
-  return cuda_status(launch_score_topk_simt(D, S, qi, kbar, sel, status_word(workspace), (cudaStream_t)stream));
+  if (workspace_bytes < kStatusBytes + scratch_need(D, S)) return QSA_ERR_INVALID_ARG;
+  return score_dispatch(D, S, qi, kbar, sel, workspace, (cudaStream_t)stream);
 }
 
 qsa_status_t qsa_sparse_attn(const qsa_config_t *cfg, const void *q, const void *k, const void *v,
@@ -273,7 +317,7 @@ qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensor
     s = cuda_status(launch_compress(D, S, t->ki_cache, nullptr, t->kbar_cache, t->kbar_blocks,
                                     status, st));
     if (s != QSA_OK) return s;
-    s = cuda_status(launch_score_topk_simt(D, S, t->qi, t->kbar_cache, t->sel, status, st));
+    s = score_dispatch(D, S, t->qi, t->kbar_cache, t->sel, workspace, st);
   } else {
     // The decode query sits at kv_len - 1; a null q_first tells the kernels so.
     S.q_first = nullptr;

@@ -104,38 +104,48 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // P for one 32-key quarter, stored as 16 packed bf16 pairs at TMEM column `col`:
-// p = 2^(s * sl2 - m) for keys below `lim`, 0 from there on.
+// p = 2^(s * sl2 - m) for keys below `lim`, 0 from there on. The scaled logits and
+// the running sum use packed fp32 pairs.
 template <bool kAll>
 __device__ __forceinline__ float p_quarter(const uint32_t *sv, int lim, float sl2, float m, uint32_t col) {
   uint32_t pk[16];
-  float ps[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint64_t scale2 = f2_splat(sl2), negm2 = f2_splat(-m);
+  uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
   for (int u = 0; u < 32; u += 2) {
-    float p0 = ex2_approx(fmaf(__uint_as_float(sv[u]), sl2, -m));
-    float p1 = ex2_approx(fmaf(__uint_as_float(sv[u + 1]), sl2, -m));
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(sv[u], sv[u + 1]), scale2, negm2), x0, x1);
+    float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
     if (!kAll) {
       p0 = (u < lim) ? p0 : 0.f;
       p1 = (u + 1 < lim) ? p1 : 0.f;
     }
-    ps[(u >> 1) & 3] += p0 + p1;
-    pk[u >> 1] = pack_bf16x2(p0, p1);
+    const uint32_t pb = pack_bf16x2(p0, p1);
+    pk[u >> 1] = pb;
+    if ((u >> 1) & 1) acc1 = f2_add(acc1, f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
+    else acc0 = f2_add(acc0, f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
   }
   tmem_st16(col, pk);
-  return (ps[0] + ps[1]) + (ps[2] + ps[3]);
+  float s0, s1;
+  f2_unpack(f2_add(acc0, acc1), s0, s1);
+  return s0 + s1;
 }
 
-// Max of the first `lim` of 64 fp32 values, with 8 independent chains.
+// Max of the first `lim` of 32 fp32 values, three at a time in 4 independent chains.
 template <bool kAll>
-__device__ __forceinline__ float max_half(const uint32_t *sv, int lim) {
-  float mx[8];
+__device__ __forceinline__ float max_quarter(const uint32_t *sv, int lim) {
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+  for (int u = 0; u < 32; u += 8) {
 #pragma unroll
-  for (int u = 0; u < kHalf; ++u) {
-    const float x = __uint_as_float(sv[u]);
-    mx[u & 7] = fmaxf(mx[u & 7], (kAll || u < lim) ? x : -INFINITY);
+    for (int e = 0; e < 4; ++e) {
+      const int a = u + 2 * e;
+      const float xa = (kAll || a < lim) ? __uint_as_float(sv[a]) : -INFINITY;
+      const float xb = (kAll || a + 1 < lim) ? __uint_as_float(sv[a + 1]) : -INFINITY;
+      mx[e] = max3f(mx[e], xa, xb);
+    }
   }
-  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+  return max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -383,19 +393,18 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           tmem_st32(s_col, zk);
           tmem_st32(s_col + 32, zk);
         } else {
-          uint32_t sv[128];
-          if (!z0) {
-            tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          }
-          if (!z1) {
-            tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-            tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-          }
-          tmem_ld_wait();
+          // pass 1: row max over the visible keys, a 32-column quarter at a time
           float cmax = -INFINITY;
-          if (!z0) cmax = f0 ? max_half<true>(&sv[0], kHalf) : max_half<false>(&sv[0], lim[0]);
-          if (!z1) cmax = fmaxf(cmax, f1 ? max_half<true>(&sv[kHalf], kHalf) : max_half<false>(&sv[kHalf], lim[1]));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int hh = q >> 1;
+            if (hh ? z1 : z0) continue;
+            uint32_t sv[32];
+            tmem_ld32(s_col + 32 * q, sv);
+            tmem_ld_wait();
+            const int lq = lim[hh] - (q & 1) * 32;
+            cmax = fmaxf(cmax, (hh ? f1 : f0) ? max_quarter<true>(sv, 32) : max_quarter<false>(sv, lq));
+          }
           cmax *= sl2;
           bool rescale = false;
           float alpha = 1.f;
@@ -408,22 +417,24 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
               m_ref = cmax;
             }
           }
-          // P of keys 32 q .. 32 q + 31 -> columns 16 q .. 16 q + 15.
+          // pass 2: P of keys 32 q .. 32 q + 31 -> columns 16 q .. 16 q + 15. Quarter q
+          // reads S columns 32 q .. 32 q + 31, which no earlier quarter's P has overwritten.
           float psum = 0.f;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int hh = q >> 1;
-            const int lq = lim[hh] - (q & 1) * 32;  // keys of this quarter below the limit
-            const bool zero = hh ? z1 : z0, full = hh ? f1 : f0;
-            if (zero) {
+            const int lq = lim[hh] - (q & 1) * 32;
+            if (hh ? z1 : z0) {
               uint32_t zk[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) zk[e] = 0u;
               tmem_st16(s_col + 16 * q, zk);
-            } else if (full) {
-              psum += p_quarter<true>(&sv[32 * q], 32, sl2, m_ref, s_col + 16 * q);
             } else {
-              psum += p_quarter<false>(&sv[32 * q], lq, sl2, m_ref, s_col + 16 * q);
+              uint32_t sv[32];
+              tmem_ld32(s_col + 32 * q, sv);
+              tmem_ld_wait();
+              psum += (hh ? f1 : f0) ? p_quarter<true>(sv, 32, sl2, m_ref, s_col + 16 * q)
+                                     : p_quarter<false>(sv, lq, sl2, m_ref, s_col + 16 * q);
             }
           }
           if (__any_sync(0xffffffffu, rescale)) {

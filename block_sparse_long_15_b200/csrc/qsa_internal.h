@@ -67,15 +67,14 @@ void note_launch(int n = 1);
 // Remember a failed CUDA call for qsa_last_error() (what + the CUDA error text).
 void note_error(const char *what, cudaError_t e);
 
-// Raise a kernel's dynamic shared memory limit once (the attribute is sticky), so
-// that launches stay legal while a stream is being captured into a CUDA graph.
+// Raise a kernel's dynamic shared memory limit once per (device, kernel) -- the
+// attribute is sticky -- so that launches stay legal while a stream is being
+// captured into a CUDA graph. Keyed by the kernel's address: instantiations of one
+// template share a type but not their attributes.
+cudaError_t ensure_smem_for(const void *kernel, size_t bytes);
 template <typename K>
 cudaError_t ensure_smem(K kernel, size_t bytes) {
-  static size_t granted = 48 * 1024;
-  if (bytes <= granted) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) granted = bytes;
-  return e;
+  return ensure_smem_for(reinterpret_cast<const void *>(kernel), bytes);
 }
 
 // ---- launches (each returns the launch error, cudaSuccess otherwise) ----
@@ -88,6 +87,13 @@ cudaError_t launch_compress(const Dims &D, const Seqs &S, const void *ki, const 
 // Steps 2+3 (CUDA cores, fp32): scores and top-k for every query row.
 cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
                                    int32_t *sel, int *status, cudaStream_t st);
+
+// Steps 2+3 on tcgen05 tensor cores (bf16 indexer, kbar as a bf16 hi/lo pair); scratch
+// holds the hi/lo planes (score_tc_workspace bytes).
+bool score_tc_supported(const Dims &D, const Seqs &S);
+size_t score_tc_workspace(const Dims &D, const Seqs &S);
+cudaError_t launch_score_topk_tc(const Dims &D, const Seqs &S, const void *qi, const float *kbar, int32_t *sel,
+                                 void *scratch, int *status, cudaStream_t st);
 
 // The decode prologue (append the new token at kv_len - 1, compress a block it
 // completes, advance kbar_blocks; see launch_decode_append) fused with steps 2+3

@@ -1,0 +1,384 @@
+// Steps 2+3 on tcgen05 tensor cores: indexer block scores and causal top-k for a
+// tile of query tokens (Hugging Face Transformers model doc "Qwen4-Exp", intro
+// paragraph on QSA: several query heads score compressed key blocks and the most
+// relevant blocks are selected; Qwen4ExpTextConfig indexer_budget).
+//
+// s[t][j] = sum_h max(0, qi[t][h] . kbar[j]) for the 32 tokens of a tile and every
+// block j < n_c of the tile, with the MMA operands swapped so that a thread owns
+// one block: D[j][(t, h)] = kbar[j] . qi[t][h] (M = 128 blocks, N = 32 Hi (token,
+// head) pairs, K = di), then the thread sums max(0, .) over h in its own registers.
+// kbar is fp32; it enters the MMA as a bf16 pair hi = bf16(kbar), lo = bf16(kbar - hi)
+// (two accumulating passes), so the scores carry about 2^-16 relative error of kbar
+// instead of bf16's 2^-9. The tile's scores go to shared memory as fp32 bit patterns
+// (scores are >= +0, so the bit order is the value order) and each warp selects the
+// top k of a token with an exact 8-bit radix select; the ids are written ascending,
+// ties to the lower block index.
+//
+// Warps: 0 TMA producer, 1 TMEM owner and MMA issuer, 2-5 epilogue (warp w reads TMEM
+// lanes 32 (w % 4) ..), then all sixteen warps run the per-token selection.
+#include <cuda.h>
+#include <math.h>
+#include <stdio.h>
+
+#include "qsa_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace qsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTok = 32;        // query tokens per CTA
+constexpr int kCand = 128;      // blocks per candidate tile (MMA M)
+constexpr int kThreads = 512;  // warps 0-5 run the MMA pipeline, all 16 the selection
+constexpr int kMaxBlocks = 1024;  // blocks a token may score (shared-memory score rows)
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+struct ScoreParams {
+  Dims D;
+  Seqs S;
+  int32_t *sel;
+  int *status;
+  int n_tiles;  // token tiles per sequence
+  int N;        // kTok * Hi
+};
+
+// Split fp32 kbar into bf16 hi and lo planes [batch * nb_cap][di].
+__global__ void k_kbar_split(const float *__restrict__ kbar, __nv_bfloat16 *__restrict__ hi,
+                             __nv_bfloat16 *__restrict__ lo, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const float v = kbar[i];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+template <int HI>
+__global__ void __launch_bounds__(kThreads, 1)
+k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant__ CUtensorMap tm_hi,
+                const __grid_constant__ CUtensorMap tm_lo, ScoreParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const Dims &D = P.D;
+  const Seqs &S = P.S;
+  constexpr int Hi = HI;
+  const int di = D.di, N = P.N;
+  const int halves = di / 64;                       // 128-byte column groups of a row
+  const uint32_t qi_bytes = (uint32_t)N * di * 2;   // B operand: N rows (token, head)
+  const uint32_t cand_bytes = (uint32_t)kCand * di * 2;
+  uint8_t *qi_s = base;                             // [halves][N][128 B]
+  uint8_t *kb_s = base + qi_bytes;                  // [2 stages][hi, lo][halves][128][128 B]
+  uint64_t *bars = (uint64_t *)(kb_s + 4 * cand_bytes);
+  // bars: 0 q_full, 1..2 k_full[stage], 3..4 k_empty[stage], 5..6 d_full[buf], 7..8 d_empty[buf]
+  uint32_t *tmem_slot = (uint32_t *)(bars + 16);
+  int *ncs = (int *)(tmem_slot + 4);                // [kTok] candidates per token (-1: padding row)
+  uint32_t *scores = (uint32_t *)(ncs + kTok);      // [kTok][row stride]
+  int *hist = (int *)kb_s;                          // [16 warps][256], over the candidate tiles once they are dead
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, b = blockIdx.y;
+  const int r0 = tile * kTok;
+  const bool ok = seq_ok(S, b, threadIdx.x == 0 ? P.status : nullptr);
+  const int len = ok ? S.kv_len[b] : 0;
+  const int qf = seq_qfirst(S, b);
+
+  if (threadIdx.x < kTok) {
+    const int r = r0 + threadIdx.x, t = qf + r;
+    ncs[threadIdx.x] = (ok && r < S.n_q && t >= 0 && t < len) ? (t + 1) / D.B : -1;
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 9; ++i) mbar_init(&bars[i], (i >= 7) ? 4u : 1u);
+    fence_mbar_init();
+  }
+  // two accumulator buffers of N columns (a power of two >= 32)
+  const uint32_t tcols = (uint32_t)(2 * N < 32 ? 32 : 2 * N);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  int nc_max = 0;
+  for (int i = 0; i < kTok; ++i) nc_max = max(nc_max, ncs[i]);
+  const int n_ct = (nc_max + kCand - 1) / kCand;   // candidate tiles with a real block
+  const int row_stride = n_ct * kCand;
+
+  bool fail = false;
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && n_ct > 0) {
+      mbar_arrive_expect_tx(&bars[0], qi_bytes);
+      for (int hf = 0; hf < halves; ++hf)
+        tma_load_2d(&tm_qi, &bars[0], qi_s + hf * (N * 128), hf * 64, (b * S.n_q + r0) * Hi);
+      for (int ct = 0; ct < n_ct; ++ct) {
+        const int st = ct & 1;
+        if (ct >= 2 && !mbar_wait(&bars[3 + st], ((ct >> 1) & 1) ^ 1, kWaitNs)) {
+          fail = true;
+          break;
+        }
+        uint8_t *dst = kb_s + st * 2 * cand_bytes;
+        mbar_arrive_expect_tx(&bars[1 + st], 2 * cand_bytes);
+        const int y = b * S.nb_cap + ct * kCand;
+        for (int hf = 0; hf < halves; ++hf) {
+          tma_load_2d(&tm_hi, &bars[1 + st], dst + hf * (kCand * 128), hf * 64, y);
+          tma_load_2d(&tm_lo, &bars[1 + st], dst + cand_bytes + hf * (kCand * 128), hf * 64, y);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && n_ct > 0) {
+      const uint32_t idesc = idesc_bf16_f32(kCand, N, false, false);
+      fail = !mbar_wait(&bars[0], 0, kWaitNs);
+      tc_fence_after();
+      const uint32_t qa = smem_u32(qi_s);
+      for (int ct = 0; ct < n_ct && !fail; ++ct) {
+        const int st = ct & 1, buf = ct & 1;
+        if (ct >= 2 && !mbar_wait(&bars[7 + buf], ((ct >> 1) & 1) ^ 1, kWaitNs)) { fail = true; break; }
+        if (!mbar_wait(&bars[1 + st], (ct >> 1) & 1, kWaitNs)) { fail = true; break; }
+        tc_fence_after();
+        const uint32_t ka = smem_u32(kb_s + st * 2 * cand_bytes);
+        const uint32_t d = tbase + (uint32_t)(buf * N);
+        int step = 0;
+        for (int part = 0; part < 2; ++part)  // hi, then lo
+          for (int hf = 0; hf < halves; ++hf)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk, ++step)
+              mma_ss(d, sdesc_sw128(ka + part * cand_bytes + hf * (kCand * 128) + kk * 32, 16, 1024),
+                     sdesc_sw128(qa + hf * (N * 128) + kk * 32, 16, 1024), idesc, step > 0 ? 1u : 0u);
+        mma_commit(&bars[5 + buf]);
+        mma_commit(&bars[3 + st]);
+      }
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- epilogue: token scores
+    const int row = 32 * (warp & 3) + lane;  // candidate within the tile
+    const uint32_t lane_addr = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
+    for (int ct = 0; ct < n_ct; ++ct) {
+      const int buf = ct & 1;
+      const bool got = mbar_wait(&bars[5 + buf], (ct >> 1) & 1, kWaitNs);
+      if (!__all_sync(0xffffffffu, got)) { fail = true; break; }
+      tc_fence_after();
+      const int j = ct * kCand + row;
+      for (int c0 = 0; c0 < N; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + (uint32_t)(buf * N + c0), v);
+        tmem_ld_wait();
+        // columns c0 .. c0 + 31 are tokens c0 / Hi .. with Hi heads each
+#pragma unroll
+        for (int tq = 0; tq < 32 / Hi; ++tq) {
+          const int tok = c0 / Hi + tq;
+          float s = 0.f;
+#pragma unroll
+          for (int h = 0; h < Hi; ++h) {
+            const float x = __uint_as_float(v[tq * Hi + h]);
+            s += x > 0.f ? x : 0.f;
+          }
+          if (j < ncs[tok]) scores[tok * row_stride + j] = __float_as_uint(s);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[7 + buf]);
+    }
+  }
+  if (fail) record_status(P.status, QSA_ERR_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, tcols);
+  }
+
+  // ---------------------------------------------------------------- per-token top-k
+  int *wh = hist + warp * 256;
+  const unsigned lt = lanemask_lt();
+  for (int tok = warp; tok < kTok; tok += kThreads / 32) {
+    const int r = r0 + tok;
+    if (r >= S.n_q) continue;
+    int32_t *out = P.sel + ((size_t)b * S.n_q + r) * D.k;
+    const int n = ncs[tok];
+    if (n <= D.k) {  // padding row (n = -1), or every complete block kept
+      for (int i = lane; i < D.k; i += 32) out[i] = (i < n) ? i : -1;
+      continue;
+    }
+    const uint32_t *keys = scores + tok * row_stride;
+    // Bits above the highest one in which the row's keys differ are common to all
+    // keys: the radix passes start below them, 8 bits at a time, so that no pass
+    // piles every key into one histogram bin.
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j = lane; j < n; j += 32) {
+      kmin = min(kmin, keys[j]);
+      kmax = max(kmax, keys[j]);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const uint32_t diff = kmin ^ kmax;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    uint32_t pmask = top >= 31 ? 0u : (0xffffffffu << (top + 1));
+    uint32_t prefix = kmax & pmask;
+    int remaining = D.k;
+    for (int hi_bit = top; hi_bit >= 0; hi_bit -= 8) {
+      const int shift = hi_bit >= 7 ? hi_bit - 7 : 0;
+      const uint32_t dmask = (2u << (hi_bit - shift)) - 1u;
+      for (int i = lane; i < 256; i += 32) wh[i] = 0;
+      __syncwarp();
+      for (int j = lane; j < n; j += 32) {
+        const uint32_t key = keys[j];
+        if ((key & pmask) == prefix) atomicAdd(&wh[(key >> shift) & dmask], 1);
+      }
+      __syncwarp();
+      // lane L owns digits 255-8L .. 248-8L (descending)
+      int c[8], tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        c[q] = wh[255 - 8 * lane - q];
+        tot += c[q];
+      }
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - tot;
+      int digit = 0, above = 0;
+      const bool mine = excl < remaining && incl >= remaining;
+      if (mine) {
+        above = excl;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (above + c[q] >= remaining) {
+            digit = 255 - 8 * lane - q;
+            break;
+          }
+          above += c[q];
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      prefix |= (uint32_t)digit << shift;
+      pmask |= dmask << shift;
+      remaining -= above;
+      __syncwarp();
+    }
+    int base_i = 0, tie_base = 0;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < n ? keys[j] : 0u;
+      const bool gt = j < n && key > prefix;
+      const bool eq = j < n && key == prefix;
+      const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+      const bool take = gt || (eq && tie_base + __popc(eq_mask & lt) < remaining);
+      const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+      if (take) out[base_i + __popc(take_mask & lt)] = j;
+      base_i += __popc(take_mask);
+      tie_base += __popc(eq_mask);
+    }
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// 2-D bf16 map [rows][cols], 128-byte swizzle, boxes of 64 columns x box_rows.
+bool make_map2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char what[192];
+    snprintf(what, sizeof what, "tensor map [%llu rows][%llu cols] box %u rows at %p: driver error %d",
+             (unsigned long long)rows, (unsigned long long)cols, box_rows, ptr, (int)r);
+    note_error(what, cudaErrorInvalidValue);
+  }
+  return r == CUDA_SUCCESS;
+}
+
+size_t smem_bytes(const Dims &D, int nb_tile_max) {
+  const int N = kTok * D.Hi;
+  return 1024 + (size_t)N * D.di * 2 + 4 * (size_t)kCand * D.di * 2 + 16 * 8 + 16 + kTok * 4 +
+         (size_t)kTok * nb_tile_max * 4;
+}
+
+}  // namespace
+
+bool score_tc_supported(const Dims &D, const Seqs &S) {
+  const int N = kTok * D.Hi;
+  const int nb_tiles = ((S.nb_cap + kCand - 1) / kCand) * kCand;
+  return D.bf16 && (D.di == 64 || D.di == 128) && (D.Hi == 1 || D.Hi == 2 || D.Hi == 4 || D.Hi == 8) &&
+         S.nb_cap <= kMaxBlocks &&
+         smem_bytes(D, nb_tiles) <= 227 * 1024;
+}
+
+size_t score_tc_workspace(const Dims &D, const Seqs &S) {
+  return 2 * (((size_t)S.batch * S.nb_cap * D.di * 2 + 255) & ~(size_t)255);
+}
+
+cudaError_t launch_score_topk_tc(const Dims &D, const Seqs &S, const void *qi, const float *kbar, int32_t *sel,
+                                 void *scratch, int *status, cudaStream_t st) {
+  if (S.batch == 0 || S.n_q == 0) return cudaSuccess;
+  const size_t plane = ((size_t)S.batch * S.nb_cap * D.di * 2 + 255) & ~(size_t)255;
+  __nv_bfloat16 *hi = (__nv_bfloat16 *)scratch;
+  __nv_bfloat16 *lo = (__nv_bfloat16 *)((char *)scratch + plane);
+  const size_t n = (size_t)S.batch * S.nb_cap * D.di;
+  if (n > 0) {
+    note_launch();
+    k_kbar_split<<<(unsigned)min((n + 255) / 256, (size_t)4096), 256, 0, st>>>(kbar, hi, lo, n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap tq, th, tl;
+  const uint64_t rows_hl = (uint64_t)S.batch * (S.nb_cap > 0 ? S.nb_cap : 1);
+  if (!make_map2d(&tq, qi, D.di, (uint64_t)S.batch * S.n_q * D.Hi, kTok * D.Hi) ||
+      !make_map2d(&th, hi, D.di, rows_hl, kCand) || !make_map2d(&tl, lo, D.di, rows_hl, kCand))
+    return cudaErrorInvalidValue;
+  ScoreParams P;
+  P.D = D;
+  P.S = S;
+  P.sel = sel;
+  P.status = status;
+  P.n_tiles = (S.n_q + kTok - 1) / kTok;
+  P.N = kTok * D.Hi;
+  const int nb_tiles = ((S.nb_cap + kCand - 1) / kCand) * kCand;
+  const size_t smem = smem_bytes(D, nb_tiles);
+  auto kern = D.Hi == 1 ? k_score_topk_tc<1> : D.Hi == 2 ? k_score_topk_tc<2> : D.Hi == 4 ? k_score_topk_tc<4>
+                                                                                  : k_score_topk_tc<8>;
+  cudaError_t e = ensure_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  note_launch();
+  kern<<<dim3(P.n_tiles, S.batch), kThreads, smem, st>>>(tq, th, tl, P);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

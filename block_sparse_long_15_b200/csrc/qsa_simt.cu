@@ -283,18 +283,46 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
   // the byte at which the running count from the top reaches `remaining`.
   __shared__ int hist[256];
   __shared__ int s_digit, s_above;
-  uint32_t prefix = 0, pmask = 0;
+  __shared__ unsigned s_min, s_max;
+  // Bits above the highest one in which the row's keys differ are common to all
+  // keys: the radix passes start below them, 8 bits at a time, so that no pass
+  // piles every key into one histogram bin.
+  if (tid == 0) {
+    s_min = 0xffffffffu;
+    s_max = 0u;
+  }
+  __syncthreads();
+  {
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j = tid; j < n_c; j += kRowThreads) {
+      kmin = min(kmin, keys[j]);
+      kmax = max(kmax, keys[j]);
+    }
+    kmin = __reduce_min_sync(kFull, kmin);
+    kmax = __reduce_max_sync(kFull, kmax);
+    if (lane == 0) {
+      atomicMin(&s_min, kmin);
+      atomicMax(&s_max, kmax);
+    }
+  }
+  __syncthreads();
+  const uint32_t diff = s_min ^ s_max;
+  const int top = diff ? 31 - __clz(diff) : -1;
+  uint32_t pmask = top >= 31 ? 0u : (0xffffffffu << (top + 1));
+  uint32_t prefix = s_max & pmask;
   int remaining = D.k;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (int hi_bit = top; hi_bit >= 0; hi_bit -= 8) {
+    const int shift = hi_bit >= 7 ? hi_bit - 7 : 0;
+    const uint32_t dmask = (2u << (hi_bit - shift)) - 1u;
     for (int i = tid; i < 256; i += kRowThreads) hist[i] = 0;
     __syncthreads();
     for (int j = tid; j < n_c; j += kRowThreads) {
       const uint32_t key = keys[j];
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
     }
     __syncthreads();
     if (warp == 0) {
-      // lane L owns bytes 255-8L .. 248-8L (descending)
+      // lane L owns digits 255-8L .. 248-8L (descending)
       int c[8], tot = 0;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -307,7 +335,7 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
         const int y = __shfl_up_sync(kFull, incl, o);
         if (lane >= o) incl += y;
       }
-      const int excl = incl - tot;  // keys in higher bytes than this lane's range
+      const int excl = incl - tot;  // keys in higher digits than this lane's range
       if (excl < remaining && incl >= remaining) {
         int above = excl;
 #pragma unroll
@@ -323,7 +351,7 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
     }
     __syncthreads();
     prefix |= (uint32_t)s_digit << shift;
-    pmask |= 255u << shift;
+    pmask |= dmask << shift;
     remaining -= s_above;
     __syncthreads();
   }
