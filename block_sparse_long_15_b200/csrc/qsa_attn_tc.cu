@@ -273,15 +273,21 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       bool fail = !mbar_wait(&bars[kBarQ], 0, kWaitNs);
       tc_fence_after();
       int n_pv0 = 0, n_pv1 = 0;  // PVs issued per tile
+      // Shared-memory descriptors are built once; a k-step moves the start address,
+      // which is the low field of the descriptor, so it is a 64-bit add of
+      // (byte offset >> 4).
+      const uint64_t q_desc0 = sdesc_sw128(smem_u32(base + kOffQ), 16, 1024);
+      const uint64_t k_desc0 = sdesc_sw128(smem_u32(base + kOffK), 16, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(smem_u32(base + kOffV), kKVBytes / 2, 1024);
       auto issue_qk = [&](int w, int i) {
-        const uint32_t q_addr = smem_u32(base + kOffQ + w * kQBytes);
-        const uint32_t k_addr = smem_u32(base + kOffK + (i % kNK) * kKVBytes);
+        const uint64_t qd = q_desc0 + (uint64_t)((w * kQBytes) >> 4);
+        const uint64_t kd = k_desc0 + (uint64_t)(((i % kNK) * kKVBytes) >> 4);
+        const uint32_t d = tbase + (uint32_t)(w * 128);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32;
-          const uint32_t qoff = (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32;
-          mma_ss(tbase + (uint32_t)(w * 128), sdesc_sw128(q_addr + qoff, 16, 1024),
-                 sdesc_sw128(k_addr + koff, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off_q = (uint64_t)(((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4);
+          const uint64_t off_k = (uint64_t)(((kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32) >> 4);
+          mma_ss(d, qd + off_q, kd + off_k, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars[kBarSFull + w]);
       };
@@ -289,11 +295,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         const int cnt = w ? n_pv1++ : n_pv0++;
         if (!mbar_wait(&bars[kBarPFull + w], cnt & 1, kWaitNs)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(base + kOffV + (i % kNV) * kKVBytes);
+        const uint64_t vd = v_desc0 + (uint64_t)(((i % kNV) * kKVBytes) >> 4);
+        const uint32_t o = tbase + 256u + (uint32_t)(w * 128), pcol = tbase + (uint32_t)(w * 128);
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(tbase + 256u + (uint32_t)(w * 128), tbase + (uint32_t)(w * 128 + kk * 8),
-                 sdesc_sw128(v_addr + kk * 2048, kKVBytes / 2, 1024), idesc_pv, (cnt > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(o, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv, (cnt > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars[kBarPVDone + w]);
         return true;
       };
