@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "qsa_kernel_launch_count": ([], ctypes.c_uint64),
         "qsa_last_error": ([], ctypes.c_char_p),
         "qsa_sparse_attn_decode_noalloc": ([cfgp, V, V, V, V, V, V, I, I, V, V], I),
+        "qsa_selftest_wait_timeout": ([V, ctypes.c_int64, V], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -81,7 +82,8 @@ _lib = _load()
 EXPORTED = ("qsa_config_validate", "qsa_topk_blocks", "qsa_status_string", "qsa_workspace_size",
             "qsa_compress_blocks", "qsa_index_score_topk", "qsa_sparse_attn", "qsa_forward",
             "qsa_read_device_status", "qsa_abi_version", "qsa_attn_kernel_name",
-            "qsa_kernel_launch_count", "qsa_last_error", "qsa_sparse_attn_decode_noalloc")
+            "qsa_kernel_launch_count", "qsa_last_error", "qsa_sparse_attn_decode_noalloc",
+            "qsa_selftest_wait_timeout")
 
 # Size of the library's fixed decode scratch (QSA_NOALLOC_SCRATCH_BYTES in qsa.h).
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -241,6 +243,13 @@ def qsa_sparse_attn_decode_noalloc(cfg, q, k, v, sel, kv_start, kv_len, out, str
     _check(_lib.qsa_sparse_attn_decode_noalloc(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(kv_start),
                                                _p(kv_len), batch, kv_cap, _p(out), _stream(stream)),
            "qsa_sparse_attn_decode_noalloc")
+
+
+def qsa_selftest_wait_timeout(workspace, limit_ns: int = 50_000_000, stream=None):
+    """Enqueue a wait that nothing completes; it gives up after limit_ns and records
+    QSA_ERR_TIMEOUT in the workspace status word (read it with qsa_read_device_status)."""
+    _check(_lib.qsa_selftest_wait_timeout(_p(workspace), int(limit_ns), _stream(stream)),
+           "qsa_selftest_wait_timeout")
 
 
 def qsa_read_device_status(workspace: torch.Tensor, stream=None) -> int:

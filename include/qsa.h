@@ -191,6 +191,13 @@ uint64_t qsa_kernel_launch_count(void);
 /* Text of the last CUDA error this library saw on the calling thread ("" if none). */
 const char *qsa_last_error(void);
 
+/* Self-test of the bounded device waits (failure detection): enqueues one CTA that
+ * waits on a barrier nothing completes, gives up after limit_ns (1 ms .. 5 s) and
+ * records QSA_ERR_TIMEOUT in the workspace status word, exactly as a pipelined
+ * kernel does when a copy never lands. Read the result with qsa_read_device_status;
+ * the CUDA context stays usable. */
+qsa_status_t qsa_selftest_wait_timeout(void *workspace, int64_t limit_ns, qsa_stream_t stream);
+
 /* Size of the fixed device array that qsa_sparse_attn_decode_noalloc uses. */
 #define QSA_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
 
