@@ -45,12 +45,14 @@ class L2Flush:
         import torch
         self.w = torch.empty(nbytes // 4, dtype=torch.float32, device=device)
         self.r = torch.zeros(nbytes // 4, dtype=torch.float32, device=device)
-        self.sink = torch.zeros(1, dtype=torch.float32, device=device)
+        self.sink = torch.zeros((), dtype=torch.float32, device=device)
 
     def zero_(self):
         import torch
         self.w.zero_()
         torch.sum(self.r, dim=0, out=self.sink)
+
+
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
