@@ -16,14 +16,19 @@
 //               same for B, so one tile's softmax overlaps the other tile's MMAs.
 //               A tile with no row that sees a chunk skips it. MMAs run in issue
 //               order, which orders a QK after the PV that read the same columns;
-//   warps 2-5   softmax of tile A, warps 6-9 tile B (warp w reads TMEM lanes
-//               32 (w % 4) ..): tcgen05.ld of the 128-column S row, the row's mask
-//               per half (a half of a selected block is visible whole, a trailing
-//               half up to the query position, anything else not at all), online
-//               softmax with a lazily rescaled reference max, P (bf16) written
-//               into the first 64 S columns with tcgen05.st for the PV MMA (A
-//               operand from TMEM); epilogue O / l rounded to bf16.
-// TMEM (512 columns): S of tile w at 128 w, O of tile w at 256 + 128 w.
+//   warps 2-9   softmax of tile A, warps 10-17 tile B. Warp w reads TMEM lanes
+//               32 (w % 4) .. and one 64-key half of the chunk, so every row has
+//               two softmax warps, one per half: tcgen05.ld of its 64 S columns,
+//               the row's mask for the half (a half of a selected block is
+//               visible whole, a trailing half up to the query position, anything
+//               else not at all), the half's row max, swapped with the partner
+//               warp through shared memory, online softmax with a lazily rescaled
+//               reference max that both halves compute alike, P (bf16) written
+//               over the half's first 32 S columns with tcgen05.st for the PV MMA
+//               (A operand from TMEM); each half rescales and writes out its 64
+//               columns of O, and the two partial row sums meet in the epilogue.
+// TMEM (512 columns): S of tile w at 128 w, O of tile w at 256 + 128 w; P of half
+// h of tile w at 128 w + 64 h.
 // Every wait is bounded; on expiry the kernel records QSA_ERR_TIMEOUT and unwinds.
 #include <cuda.h>
 #include <math.h>
@@ -44,7 +49,7 @@ constexpr int kChunk = 128;  // keys per chunk (MMA N of S = Q K^T, K of O += P 
 constexpr int kHalf = 64;    // mask granularity (smallest block size served)
 constexpr int kNK = 2;       // K ring depth
 constexpr int kNV = 2;       // V ring depth
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;  // producer, MMA, 2 tiles x 2 halves x 4 lane groups
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
@@ -56,7 +61,9 @@ constexpr uint32_t kOffK = kOffQ + kTiles * kQBytes;
 constexpr uint32_t kOffV = kOffK + kNK * kKVBytes;
 constexpr uint32_t kOffBar = kOffV + kNV * kKVBytes;
 constexpr uint32_t kOffMisc = kOffBar + 512;
-constexpr uint32_t kOffSel = kOffMisc + 64;
+constexpr uint32_t kOffXch = kOffMisc + 64;          // [parity][tile][half][row] fp32
+constexpr uint32_t kXchBytes = 2 * kTiles * 2 * kRows * 4;
+constexpr uint32_t kOffSel = kOffXch + kXchBytes;
 constexpr uint32_t kOffBitmap = kOffSel + kSelBytes;
 
 // barrier slots
@@ -66,9 +73,10 @@ constexpr int kBarKEmpty = kBarKFull + kNK;
 constexpr int kBarVFull = kBarKEmpty + kNK;
 constexpr int kBarVEmpty = kBarVFull + kNV;
 constexpr int kBarSFull = kBarVEmpty + kNV;  // [tile]
-constexpr int kBarPFull = kBarSFull + 2;     // [tile], 4 arrivals (one per softmax warp)
+constexpr int kBarPFull = kBarSFull + 2;     // [tile], 8 arrivals (one per softmax warp)
 constexpr int kBarPVDone = kBarPFull + 2;    // [tile]
-constexpr int kNumBars = kBarPVDone + 2;
+constexpr int kBarXch = kBarPVDone + 2;      // [tile][lane group], 2 arrivals (the two halves)
+constexpr int kNumBars = kBarXch + kTiles * 4;
 static_assert(kNumBars * 8 <= 512, "barrier area");
 
 struct TcParams {
@@ -103,13 +111,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
   return __all_sync(0xffffffffu, ok);
 }
 
-// P for one 32-key quarter, stored as 16 packed bf16 pairs at TMEM column `col`:
-// p = 2^(s * sl2 - m) for keys below `lim`, 0 from there on. The scaled logits and
-// the running sum use packed fp32 pairs.
+// P for one 32-key quarter held in registers (fp32 bits), written back in place
+// over sv[0 .. 15] as 16 packed bf16 pairs: p = 2^(s * sl2 - m) for keys below
+// `lim`, 0 from there on. Pair u lands in slot u / 2 <= u, after it was read. The
+// scaled logits and the running sum use packed fp32 pairs; returns the quarter's sum.
 template <bool kAll>
-__device__ __forceinline__ float p_quarter(const uint32_t *sv, int lim, float sl2, float m, uint32_t col) {
-  uint32_t pk[16];
-  const uint64_t scale2 = f2_splat(sl2), negm2 = f2_splat(-m);
+__device__ __forceinline__ float p_quarter_regs(uint32_t (&sv)[32], int lim, uint64_t scale2, uint64_t negm2) {
   uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
   for (int u = 0; u < 32; u += 2) {
@@ -120,12 +127,10 @@ __device__ __forceinline__ float p_quarter(const uint32_t *sv, int lim, float sl
       p0 = (u < lim) ? p0 : 0.f;
       p1 = (u + 1 < lim) ? p1 : 0.f;
     }
-    const uint32_t pb = pack_bf16x2(p0, p1);
-    pk[u >> 1] = pb;
+    sv[u >> 1] = pack_bf16x2(p0, p1);
     if ((u >> 1) & 1) acc1 = f2_add(acc1, f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
     else acc0 = f2_add(acc0, f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
   }
-  tmem_st16(col, pk);
   float s0, s1;
   f2_unpack(f2_add(acc0, acc1), s0, s1);
   return s0 + s1;
@@ -183,7 +188,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   const bool sel_cached = kTiles * T * k * 4 <= (int)kSelBytes;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 4u : 1u);
+    for (int i = 0; i < kNumBars; ++i)
+      mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 8u : i >= kBarXch ? 2u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -214,10 +220,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   // Per-tile chunk sets (selected blocks and trailing ranges of the tile's tokens)
   // and a shared-memory copy of the unit's selection lists.
   if (warp >= 2 && has_work) {
+    constexpr int kSoftThreads = kThreads - 64;
     const int ts = threadIdx.x - 64;
-    for (int w = ts; w < 2 * nwords; w += 256) (w < nwords ? bm0 : bm1)[w % nwords] = 0;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    for (int e = ts; e < kTiles * T * k; e += 256) {
+    for (int w = ts; w < 2 * nwords; w += kSoftThreads) (w < nwords ? bm0 : bm1)[w % nwords] = 0;
+    asm volatile("bar.sync 1, %0;" ::"n"(kSoftThreads) : "memory");
+    for (int e = ts; e < kTiles * T * k; e += kSoftThreads) {
       const int tok = e / k, i = e - tok * k, r = r0 + tok, t = qf + r;
       if (r >= S.n_q || t < 0 || t >= len) continue;
       const int j = P.sel[((size_t)b * S.n_q + r) * k + i];
@@ -226,7 +233,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       uint32_t *bm = tok < T ? bm0 : bm1;
       for (int c = (j * B) / kChunk; c <= (j * B + B - 1) / kChunk; ++c) set_bit(bm, c);
     }
-    for (int tok = ts; tok < kTiles * T; tok += 256) {
+    for (int tok = ts; tok < kTiles * T; tok += kSoftThreads) {
       const int r = r0 + tok, t = qf + r;
       if (r >= S.n_q || t < 0 || t >= len) continue;
       const int lo = ((t + 1) / B) * B;
@@ -297,9 +304,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         tc_fence_after();
         const uint64_t vd = v_desc0 + (uint64_t)(((i % kNV) * kKVBytes) >> 4);
         const uint32_t o = tbase + 256u + (uint32_t)(w * 128), pcol = tbase + (uint32_t)(w * 128);
+        // keys 16 kk .. 16 kk + 15 of half kk / 4 sit at columns 64 (kk / 4) + 8 (kk % 4)
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(o, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv, (cnt > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(o, pcol + (kk >> 2) * 64 + (kk & 3) * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                 (cnt > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars[kBarPVDone + w]);
         return true;
       };
@@ -352,18 +361,34 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int w = (warp - 2) >> 2;  // tile
+    const int sw = warp - 2;
+    const int w = sw >> 3;         // tile
+    const int hh = (sw >> 2) & 1;  // this warp's 64-key half of every chunk, and 64 columns of O
+    const int lg = warp & 3;       // TMEM lane group
     const uint32_t *bm = w ? bm1 : bm0;
-    const int row = 32 * (warp & 3) + lane;
+    const int row = 32 * lg + lane;
     const int tok = w * T + row / G, h = row % G;
     const int r = r0 + tok, t = qf + r;
     const bool valid = has_work && r < S.n_q && t >= 0 && t < len;
     const int n_c = valid ? (t + 1) / B : 0;
     const int32_t *srow = sel_cached ? sel_s + tok * k : P.sel + ((size_t)b * S.n_q + (valid ? r : 0)) * k;
-    const uint32_t lane_addr = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
-    const uint32_t s_col = lane_addr + (uint32_t)(w * 128);
-    const uint32_t o_col = lane_addr + 256u + (uint32_t)(w * 128);
+    const uint32_t lane_addr = tbase + ((uint32_t)(32 * lg) << 16);
+    const uint32_t s_col = lane_addr + (uint32_t)(w * 128 + hh * 64);
+    const uint32_t o_col = lane_addr + 256u + (uint32_t)(w * 128 + hh * 64);
     const float sl2 = D.scale * 1.4426950408889634f;
+    float *const xch = (float *)(base + kOffXch);
+    uint64_t *const xbar = &bars[kBarXch + w * 4 + lg];
+    // Exchange number e of a per-row value with the partner warp (same rows, other
+    // half). Slots alternate by parity: a warp can be at most one exchange ahead.
+    auto swap = [&](float v, int e, float &other) -> bool {
+      float *slot = xch + ((e & 1) * kTiles + w) * 2 * kRows;
+      slot[hh * kRows + row] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+      if (!warp_wait(xbar, e & 1)) return false;
+      other = slot[(hh ^ 1) * kRows + row];
+      return true;
+    };
     float m_ref = -INFINITY, l = 0.f;
     int ptr = 0, n = 0;
     bool fail = false;
@@ -371,97 +396,83 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       for (int c = next_chunk(bm0, bm1, nwords, 0); c >= 0;
            c = next_chunk(bm0, bm1, nwords, c + 1)) {
         if (!bit_of(bm, c)) continue;
-        int lim[2] = {0, 0};
+        int lim = 0;
         if (valid) {
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int key0 = c * kChunk + hh * kHalf;
-            const int jb = key0 / B;
-            if (jb < n_c) {
-              while (ptr < k && srow[ptr] >= 0 && srow[ptr] < jb) ++ptr;
-              lim[hh] = (ptr < k && srow[ptr] == jb) ? kHalf : 0;
-            } else {
-              const int last = t - key0;
-              lim[hh] = last >= 0 ? min(last + 1, kHalf) : 0;
-            }
+          const int key0 = c * kChunk + hh * kHalf;
+          const int jb = key0 / B;
+          if (jb < n_c) {
+            while (ptr < k && srow[ptr] >= 0 && srow[ptr] < jb) ++ptr;
+            lim = (ptr < k && srow[ptr] == jb) ? kHalf : 0;
+          } else {
+            const int last = t - key0;
+            lim = last >= 0 ? min(last + 1, kHalf) : 0;
           }
         }
-        const bool z0 = __all_sync(0xffffffffu, lim[0] == 0);
-        const bool z1 = __all_sync(0xffffffffu, lim[1] == 0);
-        const bool f0 = __all_sync(0xffffffffu, lim[0] == kHalf);
-        const bool f1 = __all_sync(0xffffffffu, lim[1] == kHalf);
+        const bool z = __all_sync(0xffffffffu, lim == 0);
+        const bool f = __all_sync(0xffffffffu, lim == kHalf);
         if (!warp_wait(&bars[kBarSFull + w], n & 1)) { fail = true; break; }
         tc_fence_after();
-        if (z0 && z1) {
+        // pass 1: the half's row max over its visible keys
+        float hmax = -INFINITY;
+        if (!z) {
+          uint32_t sv0[32], sv1[32];
+          tmem_ld32(s_col, sv0);
+          tmem_ld32(s_col + 32, sv1);
+          tmem_ld_wait();
+          hmax = f ? fmaxf(max_quarter<true>(sv0, 32), max_quarter<true>(sv1, 32))
+                   : fmaxf(max_quarter<false>(sv0, lim), max_quarter<false>(sv1, lim - 32));
+        }
+        float omax = -INFINITY;
+        if (!swap(hmax, n, omax)) { fail = true; break; }
+        const float cmax = fmaxf(hmax, omax) * sl2;
+        bool rescale = false;
+        float alpha = 1.f;
+        if (cmax > -INFINITY) {  // the row sees a key in this chunk
+          if (m_ref == -INFINITY) {
+            m_ref = cmax;
+          } else if (cmax > m_ref + 8.f) {
+            rescale = true;
+            alpha = ex2_approx(m_ref - cmax);
+            m_ref = cmax;
+          }
+        }
+        // pass 2: P (bf16 pairs) over the half's first 32 S columns, once all 64 are read
+        float psum = 0.f;
+        if (z) {
           uint32_t zk[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) zk[q] = 0u;
+          for (int e = 0; e < 32; ++e) zk[e] = 0u;
           tmem_st32(s_col, zk);
-          tmem_st32(s_col + 32, zk);
         } else {
-          // pass 1: row max over the visible keys, a 32-column quarter at a time
-          float cmax = -INFINITY;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int hh = q >> 1;
-            if (hh ? z1 : z0) continue;
-            uint32_t sv[32];
-            tmem_ld32(s_col + 32 * q, sv);
-            tmem_ld_wait();
-            const int lq = lim[hh] - (q & 1) * 32;
-            cmax = fmaxf(cmax, (hh ? f1 : f0) ? max_quarter<true>(sv, 32) : max_quarter<false>(sv, lq));
-          }
-          cmax *= sl2;
-          bool rescale = false;
-          float alpha = 1.f;
-          if (lim[0] > 0 || lim[1] > 0) {
-            if (m_ref == -INFINITY) {
-              m_ref = cmax;
-            } else if (cmax > m_ref + 8.f) {
-              rescale = true;
-              alpha = ex2_approx(m_ref - cmax);
-              m_ref = cmax;
-            }
-          }
-          // pass 2: P of keys 32 q .. 32 q + 31 -> columns 16 q .. 16 q + 15. Quarter q
-          // reads S columns 32 q .. 32 q + 31, which no earlier quarter's P has overwritten.
-          float psum = 0.f;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int hh = q >> 1;
-            const int lq = lim[hh] - (q & 1) * 32;
-            if (hh ? z1 : z0) {
-              uint32_t zk[16];
-#pragma unroll
-              for (int e = 0; e < 16; ++e) zk[e] = 0u;
-              tmem_st16(s_col + 16 * q, zk);
-            } else {
-              uint32_t sv[32];
-              tmem_ld32(s_col + 32 * q, sv);
-              tmem_ld_wait();
-              psum += (hh ? f1 : f0) ? p_quarter<true>(sv, 32, sl2, m_ref, s_col + 16 * q)
-                                     : p_quarter<false>(sv, lq, sl2, m_ref, s_col + 16 * q);
-            }
-          }
-          if (__any_sync(0xffffffffu, rescale)) {
-            // The reference max moved up: scale this row's O (and l) by alpha. O is
-            // stable once this tile's previous PV has completed, and the next PV
-            // waits for this warp's arrival below.
-            if (n >= 1 && !warp_wait(&bars[kBarPVDone + w], (n - 1) & 1)) { fail = true; break; }
-            tc_fence_after();
-#pragma unroll 1
-            for (int cb = 0; cb < kD / 16; ++cb) {
-              uint32_t ov[16];
-              tmem_ld16(o_col + cb * 16, ov);
-              tmem_ld_wait();
-#pragma unroll
-              for (int q = 0; q < 16; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
-              tmem_st16(o_col + cb * 16, ov);
-            }
-            l *= alpha;
-          }
-          l += psum;
+          const uint64_t scale2 = f2_splat(sl2), negm2 = f2_splat(-m_ref);
+          uint32_t sv0[32], sv1[32];
+          tmem_ld32(s_col, sv0);
+          tmem_ld_wait();
+          psum = f ? p_quarter_regs<true>(sv0, 32, scale2, negm2) : p_quarter_regs<false>(sv0, lim, scale2, negm2);
+          tmem_ld32(s_col + 32, sv1);
+          tmem_ld_wait();
+          psum += f ? p_quarter_regs<true>(sv1, 32, scale2, negm2)
+                    : p_quarter_regs<false>(sv1, lim - 32, scale2, negm2);
+          tmem_st32_lo(s_col, sv0, sv1);
         }
+        if (__any_sync(0xffffffffu, rescale)) {
+          // The reference max moved up: scale this half of the row's O (and its part
+          // of l) by alpha. O is stable once this tile's previous PV has completed,
+          // and the next PV waits for this warp's arrival below.
+          if (n >= 1 && !warp_wait(&bars[kBarPVDone + w], (n - 1) & 1)) { fail = true; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int cb = 0; cb < 2; ++cb) {
+            uint32_t ov[32];
+            tmem_ld32(o_col + cb * 32, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
+            tmem_st32(o_col + cb * 32, ov);
+          }
+          l *= alpha;
+        }
+        l += psum;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -470,6 +481,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         if (*abort_flag) { fail = true; break; }
       }
     }
+    // the two halves' partial sums of the row
+    float l_other = 0.f;
+    if (has_work && n > 0 && !fail && !swap(l, n, l_other)) fail = true;
     if (fail) {
       record_status(P.status, QSA_ERR_TIMEOUT);
       *abort_flag = 1;
@@ -482,17 +496,18 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     }
     tc_fence_after();
     const bool write = r < S.n_q && ok;
-    __nv_bfloat16 *orow = P.out + (((size_t)b * S.n_q + (write ? r : 0)) * D.Hq + g * G + h) * kD;
-    const float inv = (valid && l > 0.f) ? 1.f / l : 0.f;
+    __nv_bfloat16 *orow = P.out + (((size_t)b * S.n_q + (write ? r : 0)) * D.Hq + g * G + h) * kD + hh * 64;
+    const float lt = l + l_other;
+    const float inv = (valid && lt > 0.f) ? 1.f / lt : 0.f;
     if (__all_sync(0xffffffffu, !have_o)) {
       if (write) {
         uint4 *o4 = (uint4 *)orow;
 #pragma unroll
-        for (int q = 0; q < kD / 8; ++q) o4[q] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < 8; ++q) o4[q] = make_uint4(0, 0, 0, 0);
       }
     } else {
 #pragma unroll 1
-      for (int cb = 0; cb < kD / 16; ++cb) {
+      for (int cb = 0; cb < 4; ++cb) {
         uint32_t ov[16];
         tmem_ld16(o_col + cb * 16, ov);
         tmem_ld_wait();

@@ -139,6 +139,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       QSA_W8(0), QSA_W8(8)
       : "memory");
 }
+// 32 consecutive columns from the first 16 registers of each of two arrays: a[0 .. 15]
+// to columns 0 .. 15, b[0 .. 15] to columns 16 .. 31.
+__device__ __forceinline__ void tmem_st32_lo(uint32_t taddr, const uint32_t (&a)[32], const uint32_t (&b)[32]) {
+  const uint32_t(&r)[32] = a;
+#define QSA_WB8(i) "r"(b[i]), "r"(b[i + 1]), "r"(b[i + 2]), "r"(b[i + 3]), "r"(b[i + 4]), "r"(b[i + 5]), \
+                   "r"(b[i + 6]), "r"(b[i + 7])
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      QSA_W8(0), QSA_W8(8), QSA_WB8(0), QSA_WB8(8)
+      : "memory");
+#undef QSA_WB8
+}
 #undef QSA_R8
 #undef QSA_W8
 
