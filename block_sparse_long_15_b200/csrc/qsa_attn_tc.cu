@@ -409,7 +409,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           }
         }
         const bool z = __all_sync(0xffffffffu, lim == 0);
-        const bool f = __all_sync(0xffffffffu, lim == kHalf);
+        // Masking per key is needed only where a lane sees part of the half (its
+        // trailing block) or the half reaches past the sequence end (the cache may
+        // hold NaN there). Otherwise each lane sees all 64 keys or none: a lane that
+        // sees none takes +inf as its reference, so its p = 2^(s - inf) is 0.
+        const bool part = __any_sync(0xffffffffu, lim > 0 && lim < kHalf) || c * kChunk + hh * kHalf + kHalf > len;
         if (!warp_wait(&bars[kBarSFull + w], n & 1)) { fail = true; break; }
         tc_fence_after();
         // pass 1: the half's row max over its visible keys
@@ -419,8 +423,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           tmem_ld32(s_col, sv0);
           tmem_ld32(s_col + 32, sv1);
           tmem_ld_wait();
-          hmax = f ? fmaxf(max_quarter<true>(sv0, 32), max_quarter<true>(sv1, 32))
-                   : fmaxf(max_quarter<false>(sv0, lim), max_quarter<false>(sv1, lim - 32));
+          if (part) {
+            hmax = fmaxf(max_quarter<false>(sv0, lim), max_quarter<false>(sv1, lim - 32));
+          } else {
+            const float mx = fmaxf(max_quarter<true>(sv0, 32), max_quarter<true>(sv1, 32));
+            hmax = lim ? mx : -INFINITY;
+          }
         }
         float omax = -INFINITY;
         if (!swap(hmax, n, omax)) { fail = true; break; }
@@ -444,15 +452,16 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           for (int e = 0; e < 32; ++e) zk[e] = 0u;
           tmem_st32(s_col, zk);
         } else {
-          const uint64_t scale2 = f2_splat(sl2), negm2 = f2_splat(-m_ref);
+          const uint64_t scale2 = f2_splat(sl2);
+          const uint64_t negm2 = f2_splat(part || lim ? -m_ref : -INFINITY);
           uint32_t sv0[32], sv1[32];
           tmem_ld32(s_col, sv0);
           tmem_ld_wait();
-          psum = f ? p_quarter_regs<true>(sv0, 32, scale2, negm2) : p_quarter_regs<false>(sv0, lim, scale2, negm2);
+          psum = part ? p_quarter_regs<false>(sv0, lim, scale2, negm2) : p_quarter_regs<true>(sv0, 32, scale2, negm2);
           tmem_ld32(s_col + 32, sv1);
           tmem_ld_wait();
-          psum += f ? p_quarter_regs<true>(sv1, 32, scale2, negm2)
-                    : p_quarter_regs<false>(sv1, lim - 32, scale2, negm2);
+          psum += part ? p_quarter_regs<false>(sv1, lim - 32, scale2, negm2)
+                       : p_quarter_regs<true>(sv1, 32, scale2, negm2);
           tmem_st32_lo(s_col, sv0, sv1);
         }
         if (__any_sync(0xffffffffu, rescale)) {
@@ -497,8 +506,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     tc_fence_after();
     const bool write = r < S.n_q && ok;
     __nv_bfloat16 *orow = P.out + (((size_t)b * S.n_q + (write ? r : 0)) * D.Hq + g * G + h) * kD + hh * 64;
+    // A row that is not a query of the sequence (left padding) may hold NaN queries,
+    // hence NaN in O: its output is written as zeros by selection, not by scaling.
     const float lt = l + l_other;
-    const float inv = (valid && lt > 0.f) ? 1.f / lt : 0.f;
+    const bool keep = valid && lt > 0.f;
+    const float inv = keep ? 1.f / lt : 0.f;
     if (__all_sync(0xffffffffu, !have_o)) {
       if (write) {
         uint4 *o4 = (uint4 *)orow;
@@ -514,7 +526,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         uint32_t pk[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          pk[q] = pack_bf16x2(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv);
+          pk[q] = keep ? pack_bf16x2(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv) : 0u;
         if (write) {
           uint4 *o4 = (uint4 *)(orow + cb * 16);
           o4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);

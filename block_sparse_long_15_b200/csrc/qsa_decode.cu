@@ -390,11 +390,11 @@ k_attn_decode_pst(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x, U = P.n_units, G = D.G;
 
-  // unit prefix sums (every CTA computes them; U is small)
-  for (int u = threadIdx.x; u < U; u += kPThreads) {
-    int t, n_c;
-    pre[u + 1] = unit_items(D, S, u / D.Hkv, t, n_c);
-  }
+  // Everything up to the grid-dependency wait below reads only the sequence
+  // geometry (kv_len, kv_start, q_first), which the kernel before this one in the
+  // stream (the decode append + selection) does not write, so with programmatic
+  // dependent launch it overlaps that kernel's tail.
+  __shared__ int s_wsum[kPThreads / 32];
   if (threadIdx.x == 0) {
     pre[0] = 0;
     s_fail = 0;
@@ -404,11 +404,41 @@ k_attn_decode_pst(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     }
     fence_mbar_init();
   }
-  __syncthreads();
-  if (threadIdx.x == 0)
-    for (int u = 0; u < U; ++u) pre[u + 1] += pre[u];
+  if (warp == kWarps && lane == 0) {
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  {
+    // unit prefix sums, every CTA for itself: each thread counts a contiguous run
+    // of units, then a scan over the threads' run totals gives each run's offset
+    const int per = (U + kPThreads - 1) / kPThreads;
+    const int u_a = min(U, (int)threadIdx.x * per), u_z = min(U, u_a + per);
+    int run = 0;
+    for (int u = u_a; u < u_z; ++u) {
+      int t, n_c;
+      const int v = unit_items(D, S, u / D.Hkv, t, n_c);
+      pre[u + 1] = v;
+      run += v;
+    }
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int acc = incl - run;
+    for (int w = 0; w < warp; ++w) acc += s_wsum[w];
+    for (int u = u_a; u < u_z; ++u) {
+      acc += pre[u + 1];
+      pre[u + 1] = acc;
+    }
+  }
   __syncthreads();
   const long long T = pre[U];
+  // sel and the cache rows appended this step come from the previous kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // padding units: CTA (u mod grid) writes their output rows as zeros
   for (int u = c; u < U; u += P.C) {
     if (pre[u + 1] != pre[u]) continue;
@@ -779,8 +809,20 @@ cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, cons
     cudaError_t e = ensure_smem(k_attn_decode_pst, smem);
     if (e != cudaSuccess) return e;
     note_launch();
-    k_attn_decode_pst<<<Q.C, kPThreads, smem, st>>>(tk, tv, Q);
-    return cudaGetLastError();
+    // Programmatic dependent launch: the kernel may start while the previous kernel
+    // in the stream finishes; it waits for that kernel's results (griddepcontrol.wait)
+    // after its prologue.
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(Q.C);
+    lc.blockDim = dim3(kPThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, k_attn_decode_pst, tk, tv, Q);
   }
   DecParams P;
   P.D = D;

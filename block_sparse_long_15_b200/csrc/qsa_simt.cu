@@ -221,6 +221,10 @@ __global__ void __launch_bounds__(kRowThreads)
 k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, int32_t *__restrict__ sel,
                  int *status, DecodeAppend A) {
   extern __shared__ float smem[];
+  // The decode attention kernel that follows is launched as a programmatic
+  // dependent: let it start its prologue now; it waits for this grid's completion
+  // before it reads anything this kernel writes.
+  if (kAppend) asm volatile("griddepcontrol.launch_dependents;");
   if (kAppend) decode_append_block<T>(D, S, A, (float *)kbar, blockIdx.y, status);
   const int HD = D.Hi * D.di;
   float *qi_s = smem;                               // [Hi*di]
