@@ -334,7 +334,6 @@ size_t smem_bytes(const Dims &D, int nb_tile_max) {
 }  // namespace
 
 bool score_tc_supported(const Dims &D, const Seqs &S) {
-  const int N = kTok * D.Hi;
   const int nb_tiles = ((S.nb_cap + kCand - 1) / kCand) * kCand;
   return D.bf16 && (D.di == 64 || D.di == 128) && (D.Hi == 1 || D.Hi == 2 || D.Hi == 4 || D.Hi == 8) &&
          S.nb_cap <= kMaxBlocks &&

@@ -157,63 +157,68 @@ __global__ void k_score_topk_simt(Dims D, Seqs S, const T *__restrict__ qi,
 constexpr int kRowThreads = 256;
 constexpr int kMaxHi = 8;  // indexer heads scored together per k̄ piece
 
-__device__ __forceinline__ int block_sum(int v, int *red) {
-  v = __reduce_add_sync(kFull, v);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  int tot = 0;
-#pragma unroll
-  for (int w = 0; w < kRowThreads / 32; ++w) tot += red[w];
-  return tot;
-}
-
-// Decode prologue for sequence b, run by one CTA: check the indexer state is in
-// step (kbar_blocks == (L-1)/B; larger means the cache was cropped, which QSA does
-// not support), append the new token at L-1, and if that completes block
-// j = L/B - 1, compress it and advance kbar_blocks. Ends with a block barrier.
+// Decode prologue for sequence b, run by one CTA: append the new token at L-1
+// and, if that completes block j = L/B - 1, compress it and advance kbar_blocks.
+// The indexer state must be in step (kbar_blocks == (L-1)/B; larger means the
+// cache was cropped, which QSA does not support). Every thread reads the sequence
+// state itself, and the new rows are loaded before anything waits on it, so the
+// global reads of the prologue overlap. A completed block's k̄ row is also left in
+// `kbar_new` (shared) for the scoring that follows in the same kernel; the caller
+// synchronises the CTA before reading it. Returns the completed block, or -1.
 template <typename T>
-__device__ void decode_append_block(const Dims &D, const Seqs &S, const DecodeAppend &A, float *kbar, int b,
-                                    int *status) {
+__device__ int decode_append_row(const Dims &D, const Seqs &S, const DecodeAppend &A, float *kbar, int b,
+                                 int *status, float *kbar_new) {
   T *k_cache = (T *)A.k_cache, *v_cache = (T *)A.v_cache, *ki_cache = (T *)A.ki_cache;
   const T *k_new = (const T *)A.k_new, *v_new = (const T *)A.v_new, *ki_new = (const T *)A.ki_new;
-  __shared__ int s_go;
-  if (threadIdx.x == 0) {
-    s_go = 0;
-    if (seq_ok(S, b, status)) {
-      const int L = S.kv_len[b];
-      const int have = A.kbar_blocks[b], need = (L - 1) / D.B;
-      if (L < 1) record_status(status, QSA_ERR_DEVICE_CHECK);
-      else if (have != need) record_status(status, have > need ? QSA_ERR_UNSUPPORTED : QSA_ERR_DEVICE_CHECK);
-      else s_go = 1;
-    }
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int HD = D.Hkv * D.d;
+  // the first two elements of this thread's share of the new K/V rows and its
+  // element of the new indexer key, in flight with the state loads
+  T kn0 = T(), vn0 = T(), kn1 = T(), vn1 = T(), kin = T();
+  if (tid < HD) {
+    kn0 = k_new[(size_t)b * HD + tid];
+    vn0 = v_new[(size_t)b * HD + tid];
   }
-  __syncthreads();
-  if (s_go) {
-    const int L = S.kv_len[b], start = seq_start(S, b);
-    const size_t pos = (size_t)start + L - 1;
-    for (int i = threadIdx.x; i < D.Hkv * D.d; i += blockDim.x) {
-      const int g = i / D.d, c = i - g * D.d;
-      const size_t dst = (((size_t)b * D.Hkv + g) * S.kv_cap + pos) * D.d + c;
-      k_cache[dst] = k_new[(size_t)b * D.Hkv * D.d + i];
-      v_cache[dst] = v_new[(size_t)b * D.Hkv * D.d + i];
-    }
-    for (int c = threadIdx.x; c < D.di; c += blockDim.x)
-      ki_cache[((size_t)b * S.kv_cap + pos) * D.di + c] = ki_new[(size_t)b * D.di + c];
-    if (L % D.B == 0) {
-      __syncthreads();
-      const int j = L / D.B - 1;
-      const T *src = ki_cache + ((size_t)b * S.kv_cap + start + (size_t)j * D.B) * D.di;
-      for (int c = threadIdx.x; c < D.di; c += blockDim.x) {
-        float acc = 0.f;
-        for (int u = 0; u < D.B; ++u) acc += to_f(src[(size_t)u * D.di + c]);
-        kbar[((size_t)b * S.nb_cap + j) * D.di + c] = acc / (float)D.B;
-      }
-      if (threadIdx.x == 0) A.kbar_blocks[b] = L / D.B;
-    }
+  if (tid + nt < HD) {
+    kn1 = k_new[(size_t)b * HD + tid + nt];
+    vn1 = v_new[(size_t)b * HD + tid + nt];
   }
-  __syncthreads();
+  if (tid < D.di) kin = ki_new[(size_t)b * D.di + tid];
+  const int start = seq_start(S, b), L = S.kv_len[b], have = A.kbar_blocks[b];
+  const bool geo = start >= 0 && L >= 1 && (long long)start + L <= (long long)S.kv_cap;
+  const int need = geo ? (L - 1) / D.B : 0;
+  if (tid == 0) {
+    if (!geo) record_status(status, QSA_ERR_DEVICE_CHECK);
+    else if (have != need) record_status(status, have > need ? QSA_ERR_UNSUPPORTED : QSA_ERR_DEVICE_CHECK);
+  }
+  if (!geo || have != need) return -1;
+  const size_t pos = (size_t)start + L - 1;
+  auto put = [&](int i, T kv, T vv) {
+    const int g = i / D.d, c = i - g * D.d;
+    const size_t dst = (((size_t)b * D.Hkv + g) * S.kv_cap + pos) * D.d + c;
+    k_cache[dst] = kv;
+    v_cache[dst] = vv;
+  };
+  if (tid < HD) put(tid, kn0, vn0);
+  if (tid + nt < HD) put(tid + nt, kn1, vn1);
+  for (int i = tid + 2 * nt; i < HD; i += nt) put(i, k_new[(size_t)b * HD + i], v_new[(size_t)b * HD + i]);
+  for (int c = tid; c < D.di; c += nt)
+    ki_cache[((size_t)b * S.kv_cap + pos) * D.di + c] = c == tid ? kin : ki_new[(size_t)b * D.di + c];
+  if (L % D.B != 0) return -1;
+  // the new token completes block j: its mean, rows in key order, the last one
+  // being the token just appended (taken from ki_new rather than re-read)
+  const int j = L / D.B - 1;
+  const T *src = ki_cache + ((size_t)b * S.kv_cap + start + (size_t)j * D.B) * D.di;
+  for (int c = tid; c < D.di; c += nt) {
+    float acc = 0.f;
+    for (int u = 0; u < D.B - 1; ++u) acc += to_f(src[(size_t)u * D.di + c]);
+    acc += to_f(c == tid ? kin : ki_new[(size_t)b * D.di + c]);
+    const float m = acc / (float)D.B;
+    kbar[((size_t)b * S.nb_cap + j) * D.di + c] = m;
+    kbar_new[c] = m;
+  }
+  if (tid == 0) A.kbar_blocks[b] = L / D.B;
+  return j;
 }
 
 template <typename T, bool kAppend>
@@ -225,14 +230,18 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
   // dependent: let it start its prologue now; it waits for this grid's completion
   // before it reads anything this kernel writes.
   if (kAppend) asm volatile("griddepcontrol.launch_dependents;");
-  if (kAppend) decode_append_block<T>(D, S, A, (float *)kbar, blockIdx.y, status);
   const int HD = D.Hi * D.di;
   float *qi_s = smem;                               // [Hi*di]
-  uint32_t *keys = (uint32_t *)(qi_s + HD);         // [nb_cap]
+  float *kbar_new = qi_s + HD;                      // [di]: k̄ of a block completed by the append
+  uint32_t *keys = (uint32_t *)(kbar_new + D.di);   // [nb_cap]
   __shared__ int red[kRowThreads / 32];
   __shared__ int wbase[kRowThreads / 32 + 1];
   const int r = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the query's indexer row: loads issued first, they depend on nothing
+  const T *src = qi + ((size_t)b * S.n_q + r) * HD;
+  for (int i = tid; i < HD; i += kRowThreads) qi_s[i] = to_f(src[i]);
+  const int j_new = kAppend ? decode_append_row<T>(D, S, A, (float *)kbar, b, status, kbar_new) : -1;
   const bool ok = seq_ok(S, b, tid == 0 ? status : nullptr);
   const int len = ok ? S.kv_len[b] : 0;
   const int t = seq_qfirst(S, b) + r;
@@ -243,14 +252,12 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
     for (int i = tid; i < D.k; i += kRowThreads) out[i] = (i < n_c) ? i : -1;
     return;
   }
-  const T *src = qi + ((size_t)b * S.n_q + r) * HD;
-  for (int i = tid; i < HD; i += kRowThreads) qi_s[i] = to_f(src[i]);
   __syncthreads();
   const float *kb = kbar + (size_t)b * S.nb_cap * D.di;
   for (int j = tid; j < n_c; j += kRowThreads) {
     // the candidate's k̄ row is read in 64-float pieces whose 16 loads are all in
     // flight together; the query heads (up to kMaxHi at a time) reuse each piece
-    const float4 *kr = (const float4 *)(kb + (size_t)j * D.di);
+    const float4 *kr = (const float4 *)(j == j_new ? kbar_new : kb + (size_t)j * D.di);
     float s = 0.f;
     for (int h0 = 0; h0 < D.Hi; h0 += kMaxHi) {
       float dot[kMaxHi];
@@ -259,7 +266,7 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
       for (int c0 = 0; c0 < D.di / 4; c0 += 16) {
         float4 kv[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) kv[c] = (c0 + c < D.di / 4) ? __ldg(&kr[c0 + c]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = 0; c < 16; ++c) kv[c] = (c0 + c < D.di / 4) ? kr[c0 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int h = 0; h < kMaxHi; ++h) {
           if (h0 + h >= D.Hi) break;
@@ -552,7 +559,7 @@ cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi,
   if (S.batch == 0 || S.n_q == 0) return cudaSuccess;
   if ((long long)S.batch * S.n_q <= 4096 && D.di % 4 == 0) {
     // few rows: one CTA per row
-    const size_t smem = sizeof(float) * ((size_t)D.Hi * D.di + S.nb_cap);
+    const size_t smem = sizeof(float) * ((size_t)D.Hi * D.di + D.di + S.nb_cap);
     if (smem <= 200 * 1024) {
       dim3 grid(S.n_q, S.batch);
       note_launch();
@@ -595,7 +602,7 @@ cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi,
 cudaError_t launch_decode_append_score(const Dims &D, const Seqs &S, const DecodeAppend &A, const void *qi,
                                        float *kbar, int32_t *sel, int *status, cudaStream_t st) {
   if (S.batch == 0) return cudaSuccess;
-  const size_t smem = sizeof(float) * ((size_t)D.Hi * D.di + S.nb_cap);
+  const size_t smem = sizeof(float) * ((size_t)D.Hi * D.di + D.di + S.nb_cap);
   if (S.n_q != 1 || D.di % 4 != 0 || smem > 200 * 1024) {
     // general path: separate prologue, then the scoring launch
     cudaError_t e = launch_decode_append(D, S, A.k_cache, A.v_cache, A.ki_cache, kbar, A.kbar_blocks, A.k_new,
