@@ -30,13 +30,29 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 // ---------------------------------------------------------------------------
-// Step 1: block compression. One warp per (sequence, block); lanes over di.
+// Step 1: block compression. One warp per (sequence, block); each lane owns
+// adjacent column pairs, so one load instruction of the warp reads a whole
+// 128-byte row (di = 64, bf16), and up to 64 rows are in flight before any is added.
 // kbar[b][j][c] = (sum_{u<B} ki[start + jB + u][c]) / B, summed in key order.
 // ---------------------------------------------------------------------------
+template <typename T> struct Pair;
+template <> struct Pair<__nv_bfloat16> {
+  typedef __nv_bfloat162 type;
+  __device__ static float lo(type v) { return __low2float(v); }
+  __device__ static float hi(type v) { return __high2float(v); }
+};
+template <> struct Pair<float> {
+  typedef float2 type;
+  __device__ static float lo(type v) { return v.x; }
+  __device__ static float hi(type v) { return v.y; }
+};
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 k_compress(Dims D, Seqs S, const T *__restrict__ ki, const int32_t *__restrict__ blocks_done,
            float *__restrict__ kbar, int32_t *__restrict__ blocks_out, int *status) {
+  typedef typename Pair<T>::type P2;
+  constexpr int kRows = sizeof(T) == 2 ? 64 : 32;  // rows loaded before they are summed
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (!seq_ok(S, b, status)) return;
@@ -44,13 +60,26 @@ k_compress(Dims D, Seqs S, const T *__restrict__ ki, const int32_t *__restrict__
   const int hi = len / D.B;
   if (blocks_out && blockIdx.x == 0 && threadIdx.x == 0) blocks_out[b] = hi;
   const int lo = blocks_done ? max(blocks_done[b], 0) : 0;
+  const int pairs = D.di / 2;
   for (int j = lo + blockIdx.x * 8 + warp; j < hi; j += gridDim.x * 8) {
-    const T *src = ki + ((size_t)b * S.kv_cap + start + (size_t)j * D.B) * D.di;
+    const P2 *src = (const P2 *)(ki + ((size_t)b * S.kv_cap + start + (size_t)j * D.B) * D.di);
     float *dst = kbar + ((size_t)b * S.nb_cap + j) * D.di;
-    for (int c = lane; c < D.di; c += 32) {
-      float acc = 0.f;
-      for (int u = 0; u < D.B; ++u) acc += to_f(src[(size_t)u * D.di + c]);
-      dst[c] = acc / (float)D.B;
+    for (int cp = lane; cp < pairs; cp += 32) {
+      float a0 = 0.f, a1 = 0.f;
+      for (int u0 = 0; u0 < D.B; u0 += kRows) {
+        P2 v[kRows];
+#pragma unroll
+        for (int u = 0; u < kRows; ++u)
+          if (u0 + u < D.B) v[u] = src[(size_t)(u0 + u) * pairs + cp];
+#pragma unroll
+        for (int u = 0; u < kRows; ++u)
+          if (u0 + u < D.B) {
+            a0 += Pair<T>::lo(v[u]);
+            a1 += Pair<T>::hi(v[u]);
+          }
+      }
+      dst[2 * cp] = a0 / (float)D.B;
+      dst[2 * cp + 1] = a1 / (float)D.B;
     }
   }
 }
