@@ -382,7 +382,7 @@ k_attn_decode_pst(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   uint64_t *full = (uint64_t *)(base + kStages * 2 * kTileBytes);  // [kStages]
   uint64_t *empty = full + kStages;                                // [kStages]
   float *mrg = (float *)(empty + kStages);                         // warp merge scratch
-  int *pre = (int *)(mrg + 2 * kWarps * 8 + kWarps * 8 * kD + kStages * 8 + 8);  // [n_units + 1]
+  int *pre = (int *)(mrg + 2 * kWarps * 8 + kWarps * 8 * kD);  // [n_units + 1]
   __shared__ int s_last, s_fail;
 
   const Dims &D = P.D;
@@ -533,7 +533,6 @@ k_attn_decode_pst(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   int u = u0, u_loaded = -1;
   bool fail = false;
   float *wm = mrg, *wl = mrg + kWarps * 8, *wo = mrg + 2 * kWarps * 8;
-  float *fw = wo + kWarps * 8 * kD;  // [kStages * 8] merge weights (reused per unit; n_parts <= ...)
   int u_t = 0, u_nc = 0, u_nsel = 0;  // geometry of the current unit
   for (long long i = lo; i < hi; ++i) {
     const int n = (int)(i - lo), st = n % kStages;
@@ -671,44 +670,42 @@ k_attn_decode_pst(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     }
     const int c_first = cta_of(pre[u], C, T), c_last = cta_of(pre[u + 1] - 1, C, T);
     const int n_parts = c_last - c_first + 1;
-    __threadfence();
+    // The barrier orders this CTA's partial writes before thread 0's release on
+    // the unit counter; the CTA that brings the count to n_parts acquires the
+    // other parts' writes and, after the next barrier, all its threads read them.
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (threadIdx.x == 0) s_last = atomicAdd(&P.done[u], 1) == n_parts - 1;
+    if (threadIdx.x == 0) {
+      int old;
+      asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;" : "=r"(old) : "l"(&P.done[u]) : "memory");
+      s_last = old == n_parts - 1;
+    }
     asm volatile("bar.sync 1, 128;" ::: "memory");
     if (s_last) {
-      __threadfence();
-      // weights 2^(m_p - m) per part and head, then O = sum_p w O_p / sum_p w l_p
-      float *ml_w = wo;  // reuse: [n_parts][G] weights, then [G] inverse sums
+      // O = sum_p 2^(m_p - m) O_p / sum_p 2^(m_p - m) l_p, merged part by part
+      // with a running max; each thread reads the (m, l) of its head and its O
+      // slice of every part at once (one round trip to L2)
       const float *ml = P.part_ml + ((size_t)u + c_first) * G * 2;
-      if (threadIdx.x < G) {
-        const int hh = threadIdx.x;
-        float mm = -INFINITY;
-        for (int pp = 0; pp < n_parts; ++pp) mm = fmaxf(mm, __ldcg(&ml[(pp * G + hh) * 2]));
-        float ll = 0.f;
-        for (int pp = 0; pp < n_parts; ++pp) {
-          const float ms = __ldcg(&ml[(pp * G + hh) * 2]);
-          const float f = (ms == -INFINITY) ? 0.f : ex2_approx(ms - mm);
-          ml_w[pp * G + hh] = f;
-          ll += f * __ldcg(&ml[(pp * G + hh) * 2 + 1]);
-        }
-        fw[hh] = ll > 0.f ? 1.f / ll : 0.f;
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
       const float4 *src = (const float4 *)(P.part + ((size_t)u + c_first) * G * kD);
       __nv_bfloat16 *orow = P.out + ((size_t)b * S.n_q * D.Hq + (size_t)g * G) * kD;
       for (int e4 = threadIdx.x; e4 < G * kD / 4; e4 += kWarps * 32) {
         const int hh = (e4 * 4) / kD;
+        float m_run = -INFINITY, l_run = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
         for (int pp = 0; pp < n_parts; ++pp) {
+          const float ms = __ldcg(&ml[(pp * G + hh) * 2]), ls = __ldcg(&ml[(pp * G + hh) * 2 + 1]);
           const float4 o4 = __ldcg(&src[(size_t)pp * (G * kD / 4) + e4]);
-          const float f = ml_w[pp * G + hh];
-          acc.x = fmaf(f, o4.x, acc.x);
-          acc.y = fmaf(f, o4.y, acc.y);
-          acc.z = fmaf(f, o4.z, acc.z);
-          acc.w = fmaf(f, o4.w, acc.w);
+          if (ms == -INFINITY) continue;  // a part that saw no key of this head
+          const float m_new = fmaxf(m_run, ms);
+          const float a = ex2_approx(m_run - m_new), f = ex2_approx(ms - m_new);
+          acc.x = fmaf(f, o4.x, acc.x * a);
+          acc.y = fmaf(f, o4.y, acc.y * a);
+          acc.z = fmaf(f, o4.z, acc.z * a);
+          acc.w = fmaf(f, o4.w, acc.w * a);
+          l_run = fmaf(f, ls, l_run * a);
+          m_run = m_new;
         }
-        const float il = fw[hh];
+        const float il = l_run > 0.f ? 1.f / l_run : 0.f;
         uint2 pk;
         pk.x = pack_bf16x2(acc.x * il, acc.y * il);
         pk.y = pack_bf16x2(acc.z * il, acc.w * il);
@@ -804,7 +801,7 @@ cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, cons
     Q.C = min(sm_count(), kMaxCtas);
     Q.status = status;
     const size_t smem = 1024 + (size_t)kStages * 2 * kTileBytes + 2 * kStages * 8 +
-                        sizeof(float) * (2 * kWarps * 8 + kWarps * 8 * kD + kStages * 8 + 8) +
+                        sizeof(float) * (2 * kWarps * 8 + kWarps * 8 * kD) +
                         sizeof(int) * (Q.n_units + 1);
     cudaError_t e = ensure_smem(k_attn_decode_pst, smem);
     if (e != cudaSuccess) return e;

@@ -183,7 +183,7 @@ __global__ void k_score_topk_simt(Dims D, Seqs S, const T *__restrict__ qi,
 // candidates are spread over all threads, and the same exact radix select runs
 // with block-wide counts; selected ids are written in ascending order.
 // ---------------------------------------------------------------------------
-constexpr int kRowThreads = 256;
+constexpr int kRowThreads = 512;
 constexpr int kMaxHi = 8;  // indexer heads scored together per k̄ piece
 
 // Decode prologue for sequence b, run by one CTA: append the new token at L-1
@@ -267,42 +267,51 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
   __shared__ int wbase[kRowThreads / 32 + 1];
   const int r = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // the query's indexer row: loads issued first, they depend on nothing
+  // Loads that depend on nothing are issued first: the query's indexer row and
+  // the sequence state. As soon as the length is known every thread prefetches
+  // the k̄ rows of its candidates into L2, so that those DRAM reads are in flight
+  // during the decode append and the barrier below.
   const T *src = qi + ((size_t)b * S.n_q + r) * HD;
-  for (int i = tid; i < HD; i += kRowThreads) qi_s[i] = to_f(src[i]);
-  const int j_new = kAppend ? decode_append_row<T>(D, S, A, (float *)kbar, b, status, kbar_new) : -1;
-  const bool ok = seq_ok(S, b, tid == 0 ? status : nullptr);
-  const int len = ok ? S.kv_len[b] : 0;
-  const int t = seq_qfirst(S, b) + r;
-  const bool valid = ok && t >= 0 && t < len;
+  const T q0 = tid < HD ? src[tid] : T();
+  const int start0 = seq_start(S, b), len0 = S.kv_len[b], t = seq_qfirst(S, b) + r;
+  const bool geo = start0 >= 0 && len0 >= 0 && (long long)start0 + len0 <= (long long)S.kv_cap;
+  const bool valid = geo && t >= 0 && t < len0;
   const int n_c = valid ? (t + 1) / D.B : 0;
+  const float *kb = kbar + (size_t)b * S.nb_cap * D.di;
+  if (n_c > D.k)
+    for (int j = tid; j < n_c; j += kRowThreads)
+      for (int o = 0; o < D.di * 4; o += 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"((const char *)(kb + (size_t)j * D.di) + o));
+  const int j_new = kAppend ? decode_append_row<T>(D, S, A, (float *)kbar, b, status, kbar_new) : -1;
+  if (tid < HD) qi_s[tid] = to_f(q0);
+  for (int i = tid + kRowThreads; i < HD; i += kRowThreads) qi_s[i] = to_f(src[i]);
+  seq_ok(S, b, tid == 0 ? status : nullptr);  // records a bad geometry
   int32_t *out = sel + ((size_t)b * S.n_q + r) * D.k;
   if (n_c <= D.k) {
     for (int i = tid; i < D.k; i += kRowThreads) out[i] = (i < n_c) ? i : -1;
     return;
   }
   __syncthreads();
-  const float *kb = kbar + (size_t)b * S.nb_cap * D.di;
   for (int j = tid; j < n_c; j += kRowThreads) {
-    // the candidate's k̄ row is read in 64-float pieces whose 16 loads are all in
-    // flight together; the query heads (up to kMaxHi at a time) reuse each piece
     const float4 *kr = (const float4 *)(j == j_new ? kbar_new : kb + (size_t)j * D.di);
     float s = 0.f;
-    for (int h0 = 0; h0 < D.Hi; h0 += kMaxHi) {
-      float dot[kMaxHi];
+    if (D.di <= 64) {
+      // the candidate's k̄ row in registers; the query heads, up to kMaxHi at a
+      // time, reuse it
+      float4 kv[16];
 #pragma unroll
-      for (int h = 0; h < kMaxHi; ++h) dot[h] = 0.f;
-      for (int c0 = 0; c0 < D.di / 4; c0 += 16) {
-        float4 kv[16];
+      for (int c = 0; c < 16; ++c) kv[c] = (c < D.di / 4) ? kr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int h0 = 0; h0 < D.Hi; h0 += kMaxHi) {
+        float dot[kMaxHi];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) kv[c] = (c0 + c < D.di / 4) ? kr[c0 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int h = 0; h < kMaxHi; ++h) dot[h] = 0.f;
 #pragma unroll
         for (int h = 0; h < kMaxHi; ++h) {
           if (h0 + h >= D.Hi) break;
-          const float4 *qh = (const float4 *)(qi_s + (h0 + h) * D.di) + c0;
+          const float4 *qh = (const float4 *)(qi_s + (h0 + h) * D.di);
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            if (c0 + c >= D.di / 4) break;
+            if (c >= D.di / 4) break;
             const float4 a = qh[c];
             dot[h] = fmaf(a.x, kv[c].x, dot[h]);
             dot[h] = fmaf(a.y, kv[c].y, dot[h]);
@@ -310,10 +319,39 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
             dot[h] = fmaf(a.w, kv[c].w, dot[h]);
           }
         }
-      }
 #pragma unroll
-      for (int h = 0; h < kMaxHi; ++h)
-        if (h0 + h < D.Hi) s += dot[h] > 0.f ? dot[h] : 0.f;
+        for (int h = 0; h < kMaxHi; ++h)
+          if (h0 + h < D.Hi) s += dot[h] > 0.f ? dot[h] : 0.f;
+      }
+    } else {
+      // wider rows in 64-float pieces whose 16 loads are all in flight together
+      for (int h0 = 0; h0 < D.Hi; h0 += kMaxHi) {
+        float dot[kMaxHi];
+#pragma unroll
+        for (int h = 0; h < kMaxHi; ++h) dot[h] = 0.f;
+        for (int c0 = 0; c0 < D.di / 4; c0 += 16) {
+          float4 kv[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) kv[c] = (c0 + c < D.di / 4) ? kr[c0 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int h = 0; h < kMaxHi; ++h) {
+            if (h0 + h >= D.Hi) break;
+            const float4 *qh = (const float4 *)(qi_s + (h0 + h) * D.di) + c0;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              if (c0 + c >= D.di / 4) break;
+              const float4 a = qh[c];
+              dot[h] = fmaf(a.x, kv[c].x, dot[h]);
+              dot[h] = fmaf(a.y, kv[c].y, dot[h]);
+              dot[h] = fmaf(a.z, kv[c].z, dot[h]);
+              dot[h] = fmaf(a.w, kv[c].w, dot[h]);
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < kMaxHi; ++h)
+          if (h0 + h < D.Hi) s += dot[h] > 0.f ? dot[h] : 0.f;
+      }
     }
     keys[j] = __float_as_uint(s);
   }
