@@ -109,12 +109,14 @@ Seqs make_seqs(const Dims &D, const int32_t *kv_start, const int32_t *kv_len, co
 }
 
 // One query row per sequence (a decode step, or a stage call with n_q == 1) goes to
-// the split-KV decode kernel when it serves the shape; more rows go to the
-// tensor-core prefill kernel; everything else to the CUDA-core kernel.
-enum AttnKernel { kAttnSimt, kAttnTc, kAttnDecode };
+// the split-KV decode kernel when it serves the shape; more rows go to a
+// tensor-core prefill kernel: the two-tile kernel for head_dim 128, the one-tile
+// kernel for head_dim 256; everything else to the CUDA-core kernel.
+enum AttnKernel { kAttnSimt, kAttnTc, kAttnTc1, kAttnDecode };
 AttnKernel pick_attn(const Dims &D, const Seqs &S) {
   if (S.n_q == 1 && attn_decode_supported(D)) return kAttnDecode;
   if (attn_tc_supported(D)) return kAttnTc;
+  if (attn_tc1_supported(D)) return kAttnTc1;
   return kAttnSimt;
 }
 
@@ -170,6 +172,8 @@ qsa_status_t attn_dispatch(const Dims &D, const Seqs &S, const void *q, const vo
       return cuda_status(launch_attn_decode(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
     case kAttnTc:
       return cuda_status(launch_attn_tc(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
+    case kAttnTc1:
+      return cuda_status(launch_attn_tc1(D, S, q, k, v, sel, out, status_word(ws), st));
     default:
       return cuda_status(launch_attn_simt(D, S, q, k, v, sel, out, status_word(ws), st));
   }
@@ -213,6 +217,7 @@ const char *qsa_attn_kernel_name(const qsa_config_t *cfg, int32_t mode) {
   switch (pick_attn(D, S)) {
     case kAttnDecode: return "split-kv decode";
     case kAttnTc: return "tcgen05";
+    case kAttnTc1: return "tcgen05 one-tile";
     default: return "simt";
   }
 }

@@ -119,6 +119,12 @@ cudaError_t launch_attn_tc(const Dims &D, const Seqs &S, const void *q, const vo
                            const int32_t *sel, void *out, void *scratch, size_t scratch_bytes,
                            int *status, cudaStream_t st);
 
+// Step 4 on tcgen05 tensor cores, one 128-row tile per CTA with double-buffered S
+// (bf16, d = 256, G divides 128, block size a multiple of 64); no scratch.
+bool attn_tc1_supported(const Dims &D);
+cudaError_t launch_attn_tc1(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
+                            const int32_t *sel, void *out, int *status, cudaStream_t st);
+
 // Decode prologue: append the new token, check the indexer state is in step,
 // compress a just-completed block, advance kbar_blocks.
 cudaError_t launch_decode_append(const Dims &D, const Seqs &S, void *k_cache, void *v_cache,
