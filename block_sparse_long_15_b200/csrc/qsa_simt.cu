@@ -47,8 +47,10 @@ template <> struct Pair<float> {
   __device__ static float hi(type v) { return v.y; }
 };
 
+constexpr int kCompressWarps = 2;  // warps per CTA: the blocks spread over many SMs
+
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kCompressWarps * 32)
 k_compress(Dims D, Seqs S, const T *__restrict__ ki, const int32_t *__restrict__ blocks_done,
            float *__restrict__ kbar, int32_t *__restrict__ blocks_out, int *status) {
   typedef typename Pair<T>::type P2;
@@ -61,7 +63,7 @@ k_compress(Dims D, Seqs S, const T *__restrict__ ki, const int32_t *__restrict__
   if (blocks_out && blockIdx.x == 0 && threadIdx.x == 0) blocks_out[b] = hi;
   const int lo = blocks_done ? max(blocks_done[b], 0) : 0;
   const int pairs = D.di / 2;
-  for (int j = lo + blockIdx.x * 8 + warp; j < hi; j += gridDim.x * 8) {
+  for (int j = lo + blockIdx.x * kCompressWarps + warp; j < hi; j += gridDim.x * kCompressWarps) {
     const P2 *src = (const P2 *)(ki + ((size_t)b * S.kv_cap + start + (size_t)j * D.B) * D.di);
     float *dst = kbar + ((size_t)b * S.nb_cap + j) * D.di;
     for (int cp = lane; cp < pairs; cp += 32) {
@@ -603,16 +605,15 @@ k_decode_append(Dims D, Seqs S, T *__restrict__ k_cache, T *__restrict__ v_cache
 cudaError_t launch_compress(const Dims &D, const Seqs &S, const void *ki, const int32_t *blocks_done,
                             float *kbar, int32_t *blocks_out, int *status, cudaStream_t st) {
   if (S.batch == 0) return cudaSuccess;
-  const int per_cta = 8;
-  int gx = (S.nb_cap + per_cta - 1) / per_cta;
-  gx = max(1, min(gx, 1024));
+  int gx = (S.nb_cap + kCompressWarps - 1) / kCompressWarps;
+  gx = max(1, min(gx, 4096));
   dim3 grid(gx, S.batch);
   note_launch();
   if (D.bf16)
-    k_compress<__nv_bfloat16><<<grid, 256, 0, st>>>(D, S, (const __nv_bfloat16 *)ki, blocks_done, kbar,
+    k_compress<__nv_bfloat16><<<grid, kCompressWarps * 32, 0, st>>>(D, S, (const __nv_bfloat16 *)ki, blocks_done, kbar,
                                                     blocks_out, status);
   else
-    k_compress<float><<<grid, 256, 0, st>>>(D, S, (const float *)ki, blocks_done, kbar, blocks_out,
+    k_compress<float><<<grid, kCompressWarps * 32, 0, st>>>(D, S, (const float *)ki, blocks_done, kbar, blocks_out,
                                             status);
   return cudaGetLastError();
 }
