@@ -47,7 +47,7 @@ template <> struct Pair<float> {
   __device__ static float hi(type v) { return v.y; }
 };
 
-constexpr int kCompressWarps = 2;  // warps per CTA: the blocks spread over many SMs
+constexpr int kCompressWarps = 8;  // warps per CTA (2 per CTA measured slower at 8K)
 
 template <typename T>
 __global__ void __launch_bounds__(kCompressWarps * 32)
