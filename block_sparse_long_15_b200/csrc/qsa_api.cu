@@ -164,12 +164,14 @@ qsa_status_t score_dispatch(const Dims &D, const Seqs &S, const void *qi, const 
 }
 
 qsa_status_t attn_dispatch(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
-                           const int32_t *sel, void *out, void *ws, size_t ws_bytes, cudaStream_t st) {
+                           const int32_t *sel, void *out, void *ws, size_t ws_bytes, cudaStream_t st,
+                           bool pdl = false) {
   char *scratch = (char *)ws + kStatusBytes;
   const size_t scratch_bytes = ws_bytes - kStatusBytes;
   switch (pick_attn(D, S)) {
     case kAttnDecode:
-      return cuda_status(launch_attn_decode(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
+      return cuda_status(
+          launch_attn_decode(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st, pdl));
     case kAttnTc:
       return cuda_status(launch_attn_tc(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
     case kAttnTc1:
@@ -182,6 +184,36 @@ qsa_status_t attn_dispatch(const Dims &D, const Seqs &S, const void *q, const vo
 }  // namespace
 
 qsa_status_t qsa::resolve_config(const qsa_config_t *cfg, Dims *D) { return resolve(cfg, D); }
+
+// ---------------------------------------------------------------- cache offloading
+namespace {
+struct StagingLayout {
+  size_t k_off, v_off, sel_off, len_off, total;
+};
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+StagingLayout staging_layout(const Dims &D, int batch) {
+  const size_t esz = D.bf16 ? 2 : 4;
+  const size_t kv = round256((size_t)batch * D.Hkv * offload_cap(D) * D.d * esz);
+  StagingLayout L;
+  L.k_off = 0;
+  L.v_off = kv;
+  L.sel_off = 2 * kv;
+  L.len_off = L.sel_off + round256((size_t)batch * D.k * sizeof(int32_t));
+  L.total = L.len_off + round256((size_t)batch * sizeof(int32_t));
+  return L;
+}
+// The device address of a cache the caller keeps in host memory: page-locked host
+// memory (or device memory) is reachable from kernels, pageable memory is not.
+void *device_view(void *p) {
+  cudaPointerAttributes a;
+  if (!p || cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type == cudaMemoryTypeUnregistered) return nullptr;
+  return a.devicePointer;
+}
+}  // namespace
 
 extern "C" {
 
@@ -330,7 +362,63 @@ qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensor
     s = cuda_status(launch_decode_append_score(D, S, A, t->qi, t->kbar_cache, t->sel, status, st));
   }
   if (s != QSA_OK) return s;
-  return attn_dispatch(D, S, t->q, t->k_cache, t->v_cache, t->sel, t->out, workspace, workspace_bytes, st);
+  // In decode the kernel before the attention is this step's append/selection, which
+  // writes none of the lengths the attention's prologue reads: it may overlap it.
+  return attn_dispatch(D, S, t->q, t->k_cache, t->v_cache, t->sel, t->out, workspace, workspace_bytes, st,
+                       mode == QSA_DECODE);
+}
+
+
+qsa_status_t qsa_offload_staging_size(const qsa_config_t *cfg, int32_t batch, size_t *bytes) {
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if (!bytes || batch < 0) return QSA_ERR_INVALID_ARG;
+  *bytes = staging_layout(D, batch).total;
+  return QSA_OK;
+}
+
+qsa_status_t qsa_decode_offload(const qsa_config_t *cfg, const qsa_tensors_t *t, void *staging,
+                                size_t staging_bytes, void *workspace, size_t workspace_bytes,
+                                qsa_stream_t stream) {
+  g_serial_at_entry = g_error_serial;
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if (!t) return QSA_ERR_INVALID_ARG;
+  if ((s = check_sizes(D, t->batch, 1, t->kv_cap)) != QSA_OK) return s;
+  if (t->batch == 0) return QSA_OK;
+  if (t->n_q != 1 || !t->q || !t->qi || !t->ki_cache || (!t->kbar_cache && t->kv_cap / D.B > 0) ||
+      !t->kbar_blocks || !t->kv_start || !t->kv_len || !t->sel || !t->out || !t->k_new || !t->v_new ||
+      !t->ki_new || !staging || !workspace)
+    return QSA_ERR_INVALID_ARG;
+  void *k_dev = device_view(t->k_cache), *v_dev = device_view(t->v_cache);
+  if (!k_dev || !v_dev) {
+    note_error("qsa_decode_offload: k_cache / v_cache must be page-locked host memory or device memory",
+               cudaErrorInvalidValue);
+    return QSA_ERR_INVALID_ARG;
+  }
+  const void *ptrs[] = {t->q, t->qi, k_dev, v_dev, t->ki_cache, t->kbar_cache, t->sel, t->out,
+                        t->k_new, t->v_new, staging, workspace};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return QSA_ERR_INVALID_ARG;
+  const StagingLayout L = staging_layout(D, t->batch);
+  if (staging_bytes < L.total) return QSA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  Seqs S = make_seqs(D, t->kv_start, t->kv_len, nullptr, t->batch, 1, t->kv_cap);
+  char *stg = (char *)staging;
+  int32_t *sel_st = (int32_t *)(stg + L.sel_off), *len_st = (int32_t *)(stg + L.len_off);
+  Seqs S2 = make_seqs(D, nullptr, len_st, nullptr, t->batch, 1, (int)offload_cap(D));
+  if (workspace_bytes < kStatusBytes + scratch_need(D, S) || workspace_bytes < kStatusBytes + scratch_need(D, S2))
+    return QSA_ERR_INVALID_ARG;
+  int *status = status_word(workspace);
+  DecodeAppend A{k_dev, v_dev, t->ki_cache, t->kbar_blocks, t->k_new, t->v_new, t->ki_new};
+  s = cuda_status(launch_decode_append_score(D, S, A, t->qi, t->kbar_cache, t->sel, status, st));
+  if (s != QSA_OK) return s;
+  s = cuda_status(launch_offload_gather(D, S, k_dev, v_dev, t->k_new, t->v_new, t->sel, stg + L.k_off,
+                                        stg + L.v_off, sel_st, len_st, st));
+  if (s != QSA_OK) return s;
+  return attn_dispatch(D, S2, t->q, stg + L.k_off, stg + L.v_off, sel_st, t->out, workspace, workspace_bytes, st);
 }
 
 qsa_status_t qsa_read_device_status(void *workspace, qsa_stream_t stream, qsa_status_t *status) {

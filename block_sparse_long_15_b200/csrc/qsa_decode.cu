@@ -781,7 +781,7 @@ int sm_count() {
 
 cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
                                const int32_t *sel, void *out, void *scratch, size_t scratch_bytes, int *status,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool pdl) {
   if (!attn_decode_supported(D) || S.n_q != 1) return cudaErrorNotSupported;
   if (S.batch == 0) return cudaSuccess;
   if (scratch_bytes < attn_decode_workspace(D, S)) return cudaErrorInvalidValue;
@@ -806,9 +806,10 @@ cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, cons
     cudaError_t e = ensure_smem(k_attn_decode_pst, smem);
     if (e != cudaSuccess) return e;
     note_launch();
-    // Programmatic dependent launch: the kernel may start while the previous kernel
-    // in the stream finishes; it waits for that kernel's results (griddepcontrol.wait)
-    // after its prologue.
+    // With pdl, a programmatic dependent launch: the kernel may start while the
+    // previous kernel in the stream finishes; it waits for that kernel's results
+    // (griddepcontrol.wait) after its prologue. Without it, griddepcontrol.wait
+    // returns at once.
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(Q.C);
     lc.blockDim = dim3(kPThreads);
@@ -818,7 +819,7 @@ cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, cons
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = at;
-    lc.numAttrs = 1;
+    lc.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&lc, k_attn_decode_pst, tk, tv, Q);
   }
   DecParams P;

@@ -135,8 +135,22 @@ cudaError_t launch_decode_append(const Dims &D, const Seqs &S, void *k_cache, vo
 // Split-KV decode attention (one query per sequence), HBM-bound.
 bool attn_decode_supported(const Dims &D);
 size_t attn_decode_workspace(const Dims &D, const Seqs &S);
+// pdl: launch as a programmatic dependent of the previous kernel in the stream, whose
+// prologue (the unit prefix sums over kv_len, kv_start, q_first) overlaps that
+// kernel's tail. Only for a predecessor that writes none of those (the decode
+// append/selection kernel of qsa_forward).
 cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, const void *k,
                                const void *v, const int32_t *sel, void *out, void *scratch,
-                               size_t scratch_bytes, int *status, cudaStream_t st);
+                               size_t scratch_bytes, int *status, cudaStream_t st, bool pdl = false);
+
+// Cache offloading (decode with K/V in host memory): copy each sequence's attended
+// blocks -- its selection, then its trailing block, whose last row is this step's
+// token taken from k_new / v_new -- from the caches into a compact device staging
+// cache of capacity (k + 1) * B per (sequence, KV head), and write the selection
+// (0 .. n_sel - 1, -1 padded) and the lengths that address it there.
+size_t offload_cap(const Dims &D);
+cudaError_t launch_offload_gather(const Dims &D, const Seqs &S, const void *k_cache, const void *v_cache,
+                                  const void *k_new, const void *v_new, const int32_t *sel, void *k_stage,
+                                  void *v_stage, int32_t *sel_stage, int32_t *len_stage, cudaStream_t st);
 
 }  // namespace qsa

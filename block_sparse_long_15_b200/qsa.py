@@ -70,6 +70,8 @@ def _load() -> ctypes.CDLL:
         "qsa_last_error": ([], ctypes.c_char_p),
         "qsa_sparse_attn_decode_noalloc": ([cfgp, V, V, V, V, V, V, I, I, V, V], I),
         "qsa_selftest_wait_timeout": ([V, ctypes.c_int64, V], I),
+        "qsa_offload_staging_size": ([cfgp, I, P(S)], I),
+        "qsa_decode_offload": ([cfgp, P(qsa_tensors_t), V, S, V, S, V], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -83,7 +85,7 @@ EXPORTED = ("qsa_config_validate", "qsa_topk_blocks", "qsa_status_string", "qsa_
             "qsa_compress_blocks", "qsa_index_score_topk", "qsa_sparse_attn", "qsa_forward",
             "qsa_read_device_status", "qsa_abi_version", "qsa_attn_kernel_name",
             "qsa_kernel_launch_count", "qsa_last_error", "qsa_sparse_attn_decode_noalloc",
-            "qsa_selftest_wait_timeout")
+            "qsa_selftest_wait_timeout", "qsa_offload_staging_size", "qsa_decode_offload")
 
 # Size of the library's fixed decode scratch (QSA_NOALLOC_SCRATCH_BYTES in qsa.h).
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -243,6 +245,44 @@ def qsa_sparse_attn_decode_noalloc(cfg, q, k, v, sel, kv_start, kv_len, out, str
     _check(_lib.qsa_sparse_attn_decode_noalloc(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(kv_start),
                                                _p(kv_len), batch, kv_cap, _p(out), _stream(stream)),
            "qsa_sparse_attn_decode_noalloc")
+
+
+def qsa_offload_staging_size(cfg, batch: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.qsa_offload_staging_size(ctypes.byref(cfg), batch, ctypes.byref(n)), "qsa_offload_staging_size")
+    return n.value
+
+
+def alloc_offload_staging(cfg, batch: int, device=None) -> torch.Tensor:
+    """Device staging buffer for qsa_decode_offload (no initialisation needed)."""
+    return torch.empty(qsa_offload_staging_size(cfg, batch), dtype=torch.uint8, device=device or "cuda")
+
+
+def _p_host_or_device(t: torch.Tensor) -> int:
+    """Address of a contiguous tensor in host or device memory. Whether the device can
+    reach it (page-locked host memory or device memory) is the library's check."""
+    if not t.is_contiguous():
+        raise ValueError("QSA tensors must be contiguous")
+    return t.data_ptr()
+
+
+def qsa_decode_offload(cfg, t: Dict[str, torch.Tensor], staging, workspace, stream=None):
+    """The decode step of qsa_forward with t["k_cache"] and t["v_cache"] in page-locked
+    host memory (e.g. tensor.pin_memory()); everything else on the device. Only the
+    attended blocks are copied to the device, into `staging`."""
+    q = t["q"]
+    batch, n_q = q.shape[0], q.shape[1]
+    kv_cap = t["k_cache"].shape[2]
+    dt = _elem(cfg)
+    for name in ("q", "qi", "k_cache", "v_cache", "ki_cache", "out"):
+        if t[name].dtype != dt:
+            raise ValueError(f"{name}: dtype {t[name].dtype}, expected {dt}")
+    T = qsa_tensors_t(batch, n_q, kv_cap, _p(q), _p(t["qi"]), _p_host_or_device(t["k_cache"]),
+                      _p_host_or_device(t["v_cache"]), _p(t["ki_cache"]), _p(t["kbar_cache"]),
+                      _p(t["kbar_blocks"]), _p(t["k_new"]), _p(t["v_new"]), _p(t["ki_new"]),
+                      _p(t["kv_start"]), _p(t["kv_len"]), None, _p(t["sel"]), _p(t["out"]))
+    _check(_lib.qsa_decode_offload(ctypes.byref(cfg), ctypes.byref(T), _p(staging), staging.numel(),
+                                   _p(workspace), workspace.numel(), _stream(stream)), "qsa_decode_offload")
 
 
 def qsa_selftest_wait_timeout(workspace, limit_ns: int = 50_000_000, stream=None):

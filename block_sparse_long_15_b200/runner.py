@@ -81,3 +81,19 @@ class QSADecode:
 
     def status(self) -> int:
         return qsa.qsa_read_device_status(self.ws)
+
+
+class QSADecodeOffload(QSADecode):
+    """QSADecode with the attention K/V cache in page-locked host memory: each call
+    appends the new token to the host cache, selects on the device and copies only
+    the attended blocks to the device staging buffer (qsa_decode_offload)."""
+
+    def __init__(self, w, inp: Dict[str, torch.Tensor], device="cuda"):
+        super().__init__(w, inp, device)
+        self.t["k_cache"] = self.t["k_cache"].cpu().pin_memory()
+        self.t["v_cache"] = self.t["v_cache"].cpu().pin_memory()
+        self.staging = qsa.alloc_offload_staging(self.cfg, self.t["q"].shape[0], device)
+
+    def __call__(self, stream=None):
+        qsa.qsa_decode_offload(self.cfg, self.t, self.staging, self.ws, stream)
+        return self.t["out"], self.t["sel"]

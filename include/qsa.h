@@ -228,6 +228,31 @@ qsa_status_t qsa_sparse_attn_decode_noalloc(const qsa_config_t *cfg, const void 
                                             const int32_t *kv_len, int32_t batch, int32_t kv_cap, void *out,
                                             qsa_stream_t stream);
 
+/* Cache offloading for decode ("Qwen4-Exp" Usage tips: the indexer state is kept
+ * apart from the attention K/V cache). The attention K/V cache lives in host memory;
+ * the indexer state (ki_cache, kbar_cache, kbar_blocks) and everything else stay on
+ * the device, and only the blocks a step attends cross the host link.
+ *
+ * qsa_offload_staging_size: bytes of the device staging buffer that
+ * qsa_decode_offload needs for `batch` sequences -- K and V of (k + 1) * B tokens per
+ * (sequence, KV head) plus the remapped selection and lengths. Caller-owned device
+ * memory, 256-byte aligned, no initialisation needed.
+ *
+ * qsa_decode_offload: the QSA_DECODE step of qsa_forward with t->k_cache and
+ * t->v_cache in page-locked host memory (cudaHostAlloc or cudaHostRegister; device
+ * memory also works). Appends k_new / v_new at kv_len - 1 in the host cache and
+ * ki_new in the device indexer cache, compresses a completed block, scores and
+ * selects on the device, copies the selected blocks and the trailing block of every
+ * (sequence, KV head) into the staging buffer, and attends there. out and sel equal
+ * what qsa_forward(QSA_DECODE) gives for the same inputs.
+ *   Returns QSA_ERR_INVALID_ARG if a cache pointer is pageable host memory (the device
+ *   cannot reach it) or the staging or workspace buffer is too small; otherwise as
+ *   qsa_forward. The workspace is sized as for qsa_forward(QSA_DECODE). */
+qsa_status_t qsa_offload_staging_size(const qsa_config_t *cfg, int32_t batch, size_t *bytes);
+qsa_status_t qsa_decode_offload(const qsa_config_t *cfg, const qsa_tensors_t *t, void *staging,
+                                size_t staging_bytes, void *workspace, size_t workspace_bytes,
+                                qsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
