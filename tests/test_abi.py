@@ -117,3 +117,39 @@ def test_sizes_beyond_limits(qsa):
 
 def test_kernel_names(qsa):
     assert qsa.qsa_attn_kernel_name(_cfg(qsa, dtype="fp32", Hq=4, Hkv=1, d=64)) == "simt"
+
+
+def test_kernel_names_by_shape(qsa):
+    # head_dim 128: the two-tile tcgen05 prefill kernel and the streaming decode kernel
+    assert qsa.qsa_attn_kernel_name(_cfg(qsa)) == "tcgen05"
+    assert qsa.qsa_attn_kernel_name(_cfg(qsa), qsa.QSA_DECODE) == "split-kv decode"
+    # head_dim 256 (the config default): the one-tile kernel for prefill and decode
+    assert qsa.qsa_attn_kernel_name(_cfg(qsa, d=256)) == "tcgen05 one-tile"
+    assert qsa.qsa_attn_kernel_name(_cfg(qsa, d=256), qsa.QSA_DECODE) == "tcgen05 one-tile"
+
+
+def test_offload_staging_size(qsa):
+    # K and V of (k + 1) * B tokens per (sequence, KV head), then the remapped
+    # selection and lengths, each section rounded up to 256 bytes
+    def r256(x):
+        return (x + 255) // 256 * 256
+    for kw, batch in ((dict(), 64), (dict(d=256), 3), (dict(Hq=32, Hkv=4, Hi=8, block=128, topk=16), 7)):
+        c = _cfg(qsa, **kw)
+        cfg = dict(Hq=16, Hkv=2, d=128, Hi=4, di=64, block=64, topk=32)
+        cfg.update(kw)
+        kv = r256(batch * cfg["Hkv"] * (cfg["topk"] + 1) * cfg["block"] * cfg["d"] * 2)
+        want = 2 * kv + r256(batch * cfg["topk"] * 4) + r256(batch * 4)
+        assert qsa.qsa_offload_staging_size(c, batch) == want
+    assert qsa.qsa_offload_staging_size(_cfg(qsa), 0) == 3 * 0
+    with pytest.raises(qsa.QSAError):
+        qsa.qsa_offload_staging_size(_cfg(qsa, indexer_kv_heads=2), 4)
+
+
+def test_offload_rejects_null_arguments_on_host(qsa):
+    lib = qsa.library()
+    c = _cfg(qsa)
+    assert lib.qsa_decode_offload(ctypes.byref(c), None, None, 0, None, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    t = qsa.qsa_tensors_t()
+    t.batch, t.n_q, t.kv_cap = 2, 1, 4096  # pointers all NULL
+    assert lib.qsa_decode_offload(ctypes.byref(c), ctypes.byref(t), None, 0, None, 0, None) == \
+        qsa.QSA_ERR_INVALID_ARG
