@@ -279,37 +279,72 @@ def load_for(seconds, fn):
 
 
 def bench_prefill_e2e(args, w, inp, p, stream):
-    """Same step through qsa_forward with pinned host inputs/outputs, copies timed."""
+    """The step through qsa_forward (the public call) from pinned host inputs to a pinned
+    host output, every copy inside the timed region. Steps run as a serving loop would:
+    two sets of device buffers, uploads on one stream, qsa_forward on another, downloads
+    on a third, so that step i + 1's upload overlaps step i's compute and download
+    (the host link is full duplex and the copy engines run beside the SMs). Every step
+    still uploads all of its inputs and reads its result back. Reported: throughput
+    (ms per step over the pipelined run) and the latency of one step run alone."""
     import torch
 
     from block_sparse_long_15_b200 import qsa
+    from block_sparse_long_15_b200.runner import QSAPrefill
     names = {"q": "q", "qi": "qi", "k": "k_cache", "v": "v_cache", "ki": "ki_cache",
              "kv_start": "kv_start", "kv_len": "kv_len", "q_first": "q_first"}
     host = {k: inp[k].contiguous().pin_memory() for k in names}
-    out_h = torch.empty(p.t["out"].shape, dtype=p.t["out"].dtype).pin_memory()
+    sets = [p, QSAPrefill(w, inp)]
+    outs = [torch.empty(p.t["out"].shape, dtype=p.t["out"].dtype).pin_memory() for _ in sets]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = outs[0].numel() * outs[0].element_size()
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    free = [None, None]  # per buffer set: event after its last download
 
-    def step():
-        for k, dst in names.items():
-            p.t[dst].copy_(host[k], non_blocking=True)
-        qsa.qsa_forward(p.cfg, qsa.QSA_PREFILL, p.t, p.ws)
-        out_h.copy_(p.t["out"], non_blocking=True)
+    def step(i):
+        k = i % 2
+        x, o = sets[k], outs[k]
+        if free[k] is not None:
+            s_in.wait_event(free[k])
+        with torch.cuda.stream(s_in):
+            for name, dst in names.items():
+                x.t[dst].copy_(host[name], non_blocking=True)
+            up = torch.cuda.Event()
+            up.record(s_in)
+        s_run.wait_event(up)
+        qsa.qsa_forward(x.cfg, qsa.QSA_PREFILL, x.t, x.ws, s_run)
+        done = torch.cuda.Event()
+        done.record(s_run)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            o.copy_(x.t["out"], non_blocking=True)
+            free[k] = torch.cuda.Event()
+            free[k].record(s_out)
 
-    for _ in range(max(2, args.warmup)):
-        step()
+    for i in range(max(2, args.warmup)):
+        step(i)
     torch.cuda.synchronize()
+    # latency of one step alone
+    lat = []
+    for i in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s_in)
+        step(i)
+        b.record(s_out)
+        torch.cuda.synchronize()
+        lat.append(a.elapsed_time(b))
+    # throughput of the pipelined loop
     n = max(5, args.steps // 2)
-    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s_in)
     for i in range(n):
-        e0[i].record()
-        step()
-        e1[i].record()
+        step(i)
+    s_in.wait_stream(s_out)
+    b.record(s_in)
     torch.cuda.synchronize()
-    assert qsa.qsa_read_device_status(p.ws) == qsa.QSA_OK
-    ms = statistics.mean(a.elapsed_time(b) for a, b in zip(e0, e1))
-    return dict(ms=ms, h2d=h2d, d2h=d2h)
+    for x in sets:
+        assert qsa.qsa_read_device_status(x.ws) == qsa.QSA_OK
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    return dict(ms=a.elapsed_time(b) / n, h2d=h2d, d2h=d2h, latency_ms=statistics.median(lat))
 
 
 def decode_kernel_bytes(w, inp):
@@ -498,7 +533,8 @@ def main(argv=None):
         e = r["e2e"]
         e_ms, e_val = aggregate(e["ms"], real_rows(inp), info)
         out["e2e"] = {"value": e_val, "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
-                      "d2h_bytes_per_step": e["d2h"], "ms_per_step": e_ms}
+                      "d2h_bytes_per_step": e["d2h"], "ms_per_step": e_ms, "pipelined": True,
+                      "latency_ms": e["latency_ms"]}
     if not args.no_decode:
         wd = W.WORKLOADS[args.decode_workload]
         dec = bench_decode(args, wd, info, peaks)
