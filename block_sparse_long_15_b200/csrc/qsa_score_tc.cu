@@ -227,7 +227,42 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
     uint32_t pmask = top >= 31 ? 0u : (0xffffffffu << (top + 1));
     uint32_t prefix = kmax & pmask;
     int remaining = D.k;
-    for (int hi_bit = top; hi_bit >= 0; hi_bit -= 8) {
+    // Once the keys still matching the prefix are at most 32, the rest is settled in
+    // registers: they are gathered one per lane, sorted descending (bitonic, across
+    // the warp), and the remaining-th of them is the k-th largest key; the keys above
+    // it among them leave `remaining` ties to take.
+    auto settle = [&]() {
+      __syncwarp();
+      int base = 0;
+      for (int j0 = 0; j0 < n; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t key = j < n ? keys[j] : 0u;
+        const bool cand = j < n && (key & pmask) == prefix;
+        const unsigned m = __ballot_sync(0xffffffffu, cand);
+        if (cand) wh[base + __popc(m & lt)] = (int)key;
+        base += __popc(m);
+      }
+      __syncwarp();
+      uint32_t v = lane < base ? (uint32_t)wh[lane] : 0u;
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const uint32_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+          // descending runs where (lane & size) == 0, ascending otherwise; the last
+          // merge (size 32) leaves the whole warp descending
+          const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
+          v = keep_max ? max(v, o) : min(v, o);
+        }
+      }
+      const uint32_t val = __shfl_sync(0xffffffffu, v, remaining - 1);
+      remaining -= __popc(__ballot_sync(0xffffffffu, lane < base && v > val));
+      prefix = val;
+      pmask = 0xffffffffu;
+      __syncwarp();
+    };
+    if (top >= 0 && n <= 32) settle();
+    for (int hi_bit = top; hi_bit >= 0 && pmask != 0xffffffffu; hi_bit -= 8) {
       const int shift = hi_bit >= 7 ? hi_bit - 7 : 0;
       const uint32_t dmask = (2u << (hi_bit - shift)) - 1u;
       for (int i = lane; i < 256; i += 32) wh[i] = 0;
@@ -251,7 +286,7 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
         if (lane >= o) incl += y;
       }
       const int excl = incl - tot;
-      int digit = 0, above = 0;
+      int digit = 0, above = 0, cnt = 0;
       const bool mine = excl < remaining && incl >= remaining;
       if (mine) {
         above = excl;
@@ -259,6 +294,7 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
         for (int q = 0; q < 8; ++q) {
           if (above + c[q] >= remaining) {
             digit = 255 - 8 * lane - q;
+            cnt = c[q];
             break;
           }
           above += c[q];
@@ -267,10 +303,12 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
       const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
       digit = __shfl_sync(0xffffffffu, digit, src);
       above = __shfl_sync(0xffffffffu, above, src);
+      cnt = __shfl_sync(0xffffffffu, cnt, src);
       prefix |= (uint32_t)digit << shift;
       pmask |= dmask << shift;
       remaining -= above;
       __syncwarp();
+      if (shift > 0 && cnt <= 32) settle();
     }
     int base_i = 0, tie_base = 0;
     for (int j0 = 0; j0 < n; j0 += 32) {
