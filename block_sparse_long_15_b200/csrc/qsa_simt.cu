@@ -362,7 +362,8 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
   // keys that match the prefix found so far per value of the next byte, then keep
   // the byte at which the running count from the top reaches `remaining`.
   __shared__ int hist[256];
-  __shared__ int s_digit, s_above;
+  __shared__ int s_digit, s_above, s_cnt, s_ncand;
+  __shared__ uint32_t s_cand[32], s_val;
   __shared__ unsigned s_min, s_max;
   // Bits above the highest one in which the row's keys differ are common to all
   // keys: the radix passes start below them, 8 bits at a time, so that no pass
@@ -423,6 +424,7 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
           if (above + c[q] >= remaining) {
             s_digit = 255 - 8 * lane - q;
             s_above = above;
+            s_cnt = c[q];
             break;
           }
           above += c[q];
@@ -433,7 +435,45 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
     prefix |= (uint32_t)s_digit << shift;
     pmask |= dmask << shift;
     remaining -= s_above;
+    const int cnt = s_cnt;
     __syncthreads();
+    if (shift > 0 && cnt <= 32) {
+      // The k-th largest key lies among the at most 32 keys still matching the
+      // prefix: gather them, sort them across warp 0 (bitonic, descending) and read
+      // the remaining-th; the keys above it among them leave `remaining` ties.
+      if (tid == 0) s_ncand = 0;
+      __syncthreads();
+      for (int j = tid; j < n_c; j += kRowThreads) {
+        const uint32_t key = keys[j];
+        if ((key & pmask) == prefix) s_cand[atomicAdd(&s_ncand, 1)] = key;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int nc = s_ncand;
+        uint32_t v = lane < nc ? s_cand[lane] : 0u;
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint32_t o = __shfl_xor_sync(kFull, v, stride);
+            const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
+            v = keep_max ? max(v, o) : min(v, o);
+          }
+        }
+        const uint32_t val = __shfl_sync(kFull, v, remaining - 1);
+        const int gt = __popc(__ballot_sync(kFull, lane < nc && v > val));
+        if (lane == 0) {
+          s_val = val;
+          s_above = gt;
+        }
+      }
+      __syncthreads();
+      prefix = s_val;
+      pmask = 0xffffffffu;
+      remaining -= s_above;
+      __syncthreads();
+      break;
+    }
   }
   // ascending compaction: chunks of kRowThreads consecutive ids in thread order
   const unsigned lt = lanemask_lt();
