@@ -180,7 +180,10 @@ qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensor
 qsa_status_t qsa_read_device_status(void *workspace, qsa_stream_t stream, qsa_status_t *status);
 
 /* Library ABI version (QSA_ABI_VERSION) and the name of the kernel family that
- * qsa_sparse_attn would launch for this config ("tcgen05" or "simt"). */
+ * qsa_sparse_attn would launch for this config in this mode (QSA_PREFILL: many query
+ * rows; QSA_DECODE: one row per sequence): "tcgen05" (head_dim 128), "tcgen05
+ * one-tile" (head_dim 256), "split-kv decode" (decode, head_dim 128, B = 64, G <= 8)
+ * or "simt" (fp32 and every other shape). */
 int32_t qsa_abi_version(void);
 const char *qsa_attn_kernel_name(const qsa_config_t *cfg, int32_t mode);
 
