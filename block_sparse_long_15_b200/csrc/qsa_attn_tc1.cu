@@ -29,7 +29,6 @@
 #include <stdio.h>
 
 #include "qsa_internal.h"
-#include "qsa_tmap.h"
 #include "sm100_ptx.cuh"
 
 namespace qsa {
@@ -472,13 +471,35 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 }
 
 // ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
 // 3-D bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
               uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2) {
-  const uint64_t dims[3] = {d0, d1, d2};
-  const uint64_t strides[2] = {stride1_bytes, stride2_bytes};
-  const uint32_t box[3] = {b0, b1, b2};
-  return encode_tmap_bf16(m, ptr, 3, dims, strides, box) == CUDA_SUCCESS;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D_>
@@ -488,7 +509,7 @@ cudaError_t launch_d(const Dims &D, const Seqs &S, const void *q, const void *k,
   CUtensorMap tq, tk, tv;
   const uint64_t rows_q = (uint64_t)S.batch * S.n_q;
   const int T = kRows / D.G;
-  if (!tmap_available()) {
+  if (!encode_fn()) {
     note_error("cuTensorMapEncodeTiled entry point", cudaErrorNotSupported);
     return cudaErrorNotSupported;
   }

@@ -18,11 +18,9 @@
 #include <math.h>
 #include <stdio.h>
 
-#include <atomic>
 #include <mutex>
 
 #include "qsa_internal.h"
-#include "qsa_tmap.h"
 #include "sm100_ptx.cuh"
 
 namespace qsa {
@@ -720,11 +718,33 @@ k_attn_decode_pst(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   if (fail) record_status(P.status, QSA_ERR_TIMEOUT);
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
 bool make_kv_map(CUtensorMap *m, const void *ptr, const Dims &D, const Seqs &S) {
-  const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)S.kv_cap, (uint64_t)S.batch * D.Hkv};
-  const uint64_t strides[2] = {(uint64_t)kD * 2, (uint64_t)S.kv_cap * kD * 2};
-  const uint32_t box[3] = {64, kBlk, 1};
-  return encode_tmap_bf16(m, ptr, 3, dims, strides, box) == CUDA_SUCCESS;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)S.kv_cap, (cuuint64_t)S.batch * D.Hkv};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)S.kv_cap * kD * 2};
+  cuuint32_t box[3] = {64, kBlk, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int max_splits_for(const Dims &D) { return (D.k + 1 + kItems - 1) / kItems; }
@@ -752,16 +772,11 @@ size_t attn_decode_workspace(const Dims &D, const Seqs &S) {
 }
 
 int sm_count() {
-  // per device, looked up once; a relaxed atomic keeps concurrent first calls benign
-  static std::atomic<int> n[64];
+  static int n[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  int v = n[dev].load(std::memory_order_relaxed);
-  if (!v) {
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-    n[dev].store(v, std::memory_order_relaxed);
-  }
-  return v;
+  if (!n[dev] && cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n[dev] = 148;
+  return n[dev];
 }
 
 cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,

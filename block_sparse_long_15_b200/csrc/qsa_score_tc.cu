@@ -21,7 +21,6 @@
 #include <stdio.h>
 
 #include "qsa_internal.h"
-#include "qsa_tmap.h"
 #include "sm100_ptx.cuh"
 
 namespace qsa {
@@ -327,12 +326,34 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
   }
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
 // 2-D bf16 map [rows][cols], 128-byte swizzle, boxes of 64 columns x box_rows.
 bool make_map2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
-  const uint64_t dims[2] = {cols, rows};
-  const uint64_t strides[1] = {cols * 2};
-  const uint32_t box[2] = {64, box_rows};
-  const CUresult r = encode_tmap_bf16(m, ptr, 2, dims, strides, box);
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     char what[192];
     snprintf(what, sizeof what, "tensor map [%llu rows][%llu cols] box %u rows at %p: driver error %d",
