@@ -64,3 +64,32 @@ def test_aggregate_two_gloo_ranks():
     for rank, ms, value in res:
         assert ms == 15.0  # the slowest rank's time
         assert value == pytest.approx(2 * 8192 / 15e-3)
+
+
+def test_ncu_traffic_voided_when_kernel_source_changes(tmp_path, monkeypatch):
+    import json
+    src = tmp_path / "kern.cu"
+    src.write_text("__global__ void k() {}\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    entry = {"kernel": "k", "source": "kern.cu", "source_sha": bench.file_sha("kern.cu"),
+             "dram_bytes_per_launch": 1234.0}
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps({"attn_prefill:w": entry}))
+    assert bench.ncu_traffic("attn_prefill:w") == 1234.0
+    assert bench.ncu_traffic("attn_prefill:other") is None
+    src.write_text("__global__ void k() { /* changed */ }\n")
+    assert bench.ncu_traffic("attn_prefill:w") is None
+
+
+def test_decode_kernel_bytes_counts_attended_tokens():
+    w = W.small_variant(W.WORKLOADS["bf16_decode_b64_l4k_32k"], seq=4096, batch=5, len_min=40, len_max=4000)
+    inp = W.make_inputs(w)
+    want = 0
+    for b in range(w.batch):
+        L = int(inp["kv_len"][b])
+        t = L - 1
+        n_c = (t + 1) // w.block
+        sel = np.array(list(range(min(n_c, w.topk))) + [-1] * max(0, w.topk - n_c), dtype=np.int32)
+        toks = len(oracle.token_set(t, w.block, sel))  # attended tokens of the decode row
+        want += toks * w.Hkv * w.d * 2 * 2 + 2 * w.Hq * w.d * 2  # K and V, then q and out (bf16)
+    assert bench.decode_kernel_bytes(w, inp) == want
