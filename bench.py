@@ -1,13 +1,18 @@
 #!/usr/bin/env python
 """Benchmark of the QSA hot path on B200.
 
-Default (N=1): bf16 prefill, batch 1, seq 8192, 16 query / 2 KV heads, head_dim
-128, 4 indexer heads of dim 64, block 64, top-k 32 (+ trailing block). A step is
-one pass of the whole path (compress -> score/top-k -> sparse attention) over
-that prompt, inputs resident in HBM, L2 flushed between steps. Also measured:
-  e2e       -- the same step through qsa_forward with pinned HOST buffers, the
-               host->device copies of the inputs and the device->host read of the
-               output inside the timed region;
+Default (N=1): the largest single-GPU workload, a batched variable-length bf16
+prefill: batch 8, padded length 16384, left pads uniform in [0, 2048], 32 query /
+4 KV heads, head_dim 128, 8 indexer heads of dim 64, block 128, top-k 16 (+ the
+trailing block). A step is one pass of the whole path (compress -> score/top-k ->
+sparse attention) over that batch, inputs resident in HBM, L2 flushed between
+steps. Also measured:
+  workloads -- the same step on the long 64K prefill (planted blocks, top-k 64) and
+               on the 8K prefill (16 / 2 heads, block 64, top-k 32), each with its
+               attention kernel's roofline;
+  e2e       -- the headline step through qsa_forward with pinned HOST buffers, the
+               host->device copy of the inputs (one copy from a pinned arena) and
+               the device->host read of the output inside the timed region;
   decode    -- one decode step for 64 sequences with caches of 4096..32768 tokens
                (CUDA-graph replay, L2 flushed between steps), plus its attention
                kernel against the HBM roofline;
@@ -63,12 +68,17 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="bf16_prefill_s8192")
+    p.add_argument("--workload", default="bf16_prefill_varlen_b8_s16384_leftpad")
+    p.add_argument("--extra-workloads", default="bf16_prefill_s65536_planted,bf16_prefill_s8192",
+                   help="comma-separated prefill workloads measured beside the headline ('' for none)")
     p.add_argument("--decode-workload", default="bf16_decode_b64_l4k_32k")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the headline workload's batch (a smaller case of the same shape, for "
+                        "profiling captures); 0 keeps the workload's own")
     return p.parse_args(argv)
 
 
@@ -209,7 +219,7 @@ def cpu_oracle_rate(w, inp, seconds, seed=0):
 
 
 # --------------------------------------------------------------------------- GPU arms
-def bench_prefill(args, w, inp, dist_info):
+def bench_prefill(args, w, inp, dist_info, with_e2e=True):
     import torch
 
     from block_sparse_long_15_b200 import qsa
@@ -262,7 +272,7 @@ def bench_prefill(args, w, inp, dist_info):
     assert qsa.qsa_read_device_status(ws) == qsa.QSA_OK
 
     e2e = None
-    if not args.no_e2e:
+    if with_e2e and not args.no_e2e:
         e2e = bench_prefill_e2e(args, w, inp, p, stream)
     return dict(step_ms=step_ms, stage_ms=stage_ms, launches=launches, clocks=clk.summary(), e2e=e2e,
                 kernel=qsa.qsa_attn_kernel_name(cfg))
@@ -278,24 +288,57 @@ def load_for(seconds, fn):
         torch.cuda.synchronize()
 
 
+class PinnedArena:
+    """Inputs of one step packed into one pinned host buffer and one device buffer of
+    the same layout (each tensor 256-byte aligned), so that a step's upload is a
+    single host->device copy."""
+
+    def __init__(self, tensors, device):
+        import torch
+        self.layout, off = {}, 0
+        for name, t in tensors.items():
+            n = t.numel() * t.element_size()
+            self.layout[name] = (off, n, t.dtype, tuple(t.shape))
+            off += (n + 255) // 256 * 256
+        self.host = torch.empty(off, dtype=torch.uint8).pin_memory()
+        for name, t in tensors.items():
+            self.view(self.host, name).copy_(t)
+        self.device = device
+        self.nbytes = off
+
+    def view(self, buf, name):
+        off, n, dt, shape = self.layout[name]
+        return buf[off:off + n].view(dt).view(shape)
+
+    def device_buffer(self):
+        import torch
+        return torch.empty(self.nbytes, dtype=torch.uint8, device=self.device)
+
+
 def bench_prefill_e2e(args, w, inp, p, stream):
     """The step through qsa_forward (the public call) from pinned host inputs to a pinned
     host output, every copy inside the timed region. Steps run as a serving loop would:
     two sets of device buffers, uploads on one stream, qsa_forward on another, downloads
     on a third, so that step i + 1's upload overlaps step i's compute and download
     (the host link is full duplex and the copy engines run beside the SMs). Every step
-    still uploads all of its inputs and reads its result back. Reported: throughput
-    (ms per step over the pipelined run) and the latency of one step run alone."""
+    still uploads all of its inputs -- one copy of the packed arena -- and reads its
+    result back. Reported: throughput (ms per step over the pipelined run) and the
+    latency of one step run alone."""
     import torch
 
     from block_sparse_long_15_b200 import qsa
     from block_sparse_long_15_b200.runner import QSAPrefill
     names = {"q": "q", "qi": "qi", "k": "k_cache", "v": "v_cache", "ki": "ki_cache",
              "kv_start": "kv_start", "kv_len": "kv_len", "q_first": "q_first"}
-    host = {k: inp[k].contiguous().pin_memory() for k in names}
-    sets = [p, QSAPrefill(w, inp)]
+    arena = PinnedArena({k: inp[k].contiguous() for k in names}, torch.cuda.current_device())
+    sets, bufs = [p, QSAPrefill(w, inp)], []
+    for x in sets:  # the buffer set's inputs become views of its device arena
+        buf = arena.device_buffer()
+        for name, dst in names.items():
+            x.t[dst] = arena.view(buf, name)
+        bufs.append(buf)
     outs = [torch.empty(p.t["out"].shape, dtype=p.t["out"].dtype).pin_memory() for _ in sets]
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    h2d = arena.nbytes
     d2h = outs[0].numel() * outs[0].element_size()
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     free = [None, None]  # per buffer set: event after its last download
@@ -306,8 +349,7 @@ def bench_prefill_e2e(args, w, inp, p, stream):
         if free[k] is not None:
             s_in.wait_event(free[k])
         with torch.cuda.stream(s_in):
-            for name, dst in names.items():
-                x.t[dst].copy_(host[name], non_blocking=True)
+            bufs[k].copy_(arena.host, non_blocking=True)
             up = torch.cuda.Event()
             up.record(s_in)
         s_run.wait_event(up)
@@ -344,7 +386,8 @@ def bench_prefill_e2e(args, w, inp, p, stream):
     for x in sets:
         assert qsa.qsa_read_device_status(x.ws) == qsa.QSA_OK
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
-    return dict(ms=a.elapsed_time(b) / n, h2d=h2d, d2h=d2h, latency_ms=statistics.median(lat))
+    return dict(ms=a.elapsed_time(b) / n, h2d=h2d, d2h=d2h, latency_ms=statistics.median(lat),
+                copies_per_step={"h2d": 1, "d2h": 1})
 
 
 def decode_kernel_bytes(w, inp):
@@ -492,6 +535,8 @@ def main(argv=None):
     n_gpus = 1 if info is None else info["world"]
     from block_sparse_long_15_b200 import workloads as W
     w = W.WORKLOADS[args.workload]
+    if args.batch > 0 and args.batch != w.batch:
+        w = w.replace(batch=args.batch, name=f"{w.name}__b{args.batch}")
     if args.impl == "reference":
         return main_reference(args, w, info, rank, n_gpus)
 
@@ -501,6 +546,61 @@ def main(argv=None):
     peaks, peak_src = load_peaks()
     inp = W.make_inputs(w)
     r = bench_prefill(args, w, inp, info)
+    head = prefill_record(w, inp, r, peaks, peak_src, info)
+    out = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": n_gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq, "num_attention_heads": w.Hq,
+                   "num_key_value_heads": w.Hkv, "head_dim": w.d, "indexer_n_heads": w.Hi,
+                   "indexer_head_dim": w.di, "indexer_compress_ratio": w.block,
+                   "indexer_budget": w.topk * w.block, "left_pad_max": w.pad_max, "seed": w.seed,
+                   "real_tokens": real_rows(inp),
+                   "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
+                   "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU"},
+        "roofline": head["roofline"],
+        "gpu_launches": r["launches"], "clocks": r["clocks"],
+    }
+    if r["e2e"]:
+        e = r["e2e"]
+        e_ms, e_val = aggregate(e["ms"], real_rows(inp), info)
+        out["e2e"] = {"value": e_val, "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
+                      "d2h_bytes_per_step": e["d2h"], "ms_per_step": e_ms, "pipelined": True,
+                      "latency_ms": e["latency_ms"], "copies_per_step": e["copies_per_step"]}
+    cpu_inp = inp if (rank == 0 and n_gpus == 1 and not args.no_cpu_baseline) else None
+    del r
+    torch.cuda.empty_cache()
+    extra = {}
+    for name in [x for x in args.extra_workloads.split(",") if x]:
+        wx = W.WORKLOADS[name]
+        ix = W.make_inputs(wx)
+        rx = bench_prefill(args, wx, ix, info, with_e2e=False)
+        rec = prefill_record(wx, ix, rx, peaks, peak_src, info)
+        rec["clocks"] = rx["clocks"]
+        rec["gpu_launches"] = rx["launches"]
+        extra[name] = rec
+        del rx, ix
+        torch.cuda.empty_cache()
+    if extra:
+        out["workloads"] = extra
+    if not args.no_decode:
+        wd = W.WORKLOADS[args.decode_workload]
+        dec = bench_decode(args, wd, info, peaks)
+        dec["us_per_step"] = max_over_ranks(dec["us_per_step"], info)
+        out["decode"] = dec
+    if cpu_inp is not None:
+        out["cpu_baseline"] = cpu_oracle_rate(w, cpu_inp, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if info is not None:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def prefill_record(w, inp, r, peaks, peak_src, info):
+    """Throughput of a prefill step and its attention kernel's roofline (selected-token
+    FLOPs only; masked tensor-core work is never counted)."""
     ms_rank = statistics.mean(r["step_ms"])
     ms, value = aggregate(ms_rank, real_rows(inp), info)
     pairs, score_pairs = attended_pairs(w, inp)
@@ -508,16 +608,8 @@ def main(argv=None):
     score_flops = 2.0 * w.Hi * w.di * score_pairs
     attn_ms = statistics.mean(r["stage_ms"][2])
     achieved = attn_flops / (attn_ms * 1e-3) / 1e12
-    out = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n_gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq, "num_attention_heads": w.Hq,
-                   "num_key_value_heads": w.Hkv, "head_dim": w.d, "indexer_n_heads": w.Hi,
-                   "indexer_head_dim": w.di, "indexer_compress_ratio": w.block,
-                   "indexer_budget": w.topk * w.block, "seed": w.seed,
-                   "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
-                   "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU"},
+    return {
+        "workload": w.name, "value": value, "unit": "tokens/s", "ms_per_step": ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"],
                      "traffic": ncu_traffic("attn_prefill:" + w.name),
@@ -527,27 +619,7 @@ def main(argv=None):
                                   "score_topk": statistics.mean(r["stage_ms"][1]),
                                   "sparse_attn": attn_ms},
                      "score_flops_per_launch": score_flops},
-        "gpu_launches": r["launches"], "clocks": r["clocks"],
     }
-    if r["e2e"]:
-        e = r["e2e"]
-        e_ms, e_val = aggregate(e["ms"], real_rows(inp), info)
-        out["e2e"] = {"value": e_val, "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
-                      "d2h_bytes_per_step": e["d2h"], "ms_per_step": e_ms, "pipelined": True,
-                      "latency_ms": e["latency_ms"]}
-    if not args.no_decode:
-        wd = W.WORKLOADS[args.decode_workload]
-        dec = bench_decode(args, wd, info, peaks)
-        dec["us_per_step"] = max_over_ranks(dec["us_per_step"], info)
-        out["decode"] = dec
-    if rank == 0 and n_gpus == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_oracle_rate(w, inp, args.cpu_seconds)
-    if rank == 0:
-        print(json.dumps(out), flush=True)
-    if info is not None:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
 
 
 def main_reference(args, w, info, rank, n_gpus):
@@ -567,7 +639,11 @@ def main_reference(args, w, info, rank, n_gpus):
     value = statistics.mean(r["value"] for r in rates)
     ms = 1e3 * real_rows(inp) / value
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n_gpus,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "ms_per_step_extrapolated": True,
+           "ms_per_step_note": (f"extrapolated: the workload's {real_rows(inp)} real query rows divided by the "
+                                "measured rows/s of the bounded samples; each timed step runs a sample only"),
+           "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq},
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": rates[0]["cores"], "kind": "oracle",

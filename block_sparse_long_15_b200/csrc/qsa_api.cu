@@ -269,7 +269,7 @@ qsa_status_t qsa_workspace_size(const qsa_config_t *cfg, int32_t mode, int32_t b
 
 qsa_status_t qsa_compress_blocks(const qsa_config_t *cfg, const void *ki, const int32_t *kv_start,
                                  const int32_t *kv_len, const int32_t *blocks_done, int32_t batch,
-                                 int32_t kv_cap, float *kbar, qsa_stream_t stream) {
+                                 int32_t kv_cap, float *kbar, int32_t *kbar_blocks, qsa_stream_t stream) {
   g_serial_at_entry = g_error_serial;
   Dims D;
   qsa_status_t s = resolve(cfg, &D);
@@ -280,7 +280,7 @@ qsa_status_t qsa_compress_blocks(const qsa_config_t *cfg, const void *ki, const 
   if (!ki || !kv_start || !kv_len || (!kbar && kv_cap / D.B > 0)) return QSA_ERR_INVALID_ARG;
   if (!aligned16(ki) || !aligned16(kbar)) return QSA_ERR_INVALID_ARG;
   Seqs S = make_seqs(D, kv_start, kv_len, nullptr, batch, 0, kv_cap);
-  return cuda_status(launch_compress(D, S, ki, blocks_done, kbar, nullptr, nullptr, (cudaStream_t)stream));
+  return cuda_status(launch_compress(D, S, ki, blocks_done, kbar, kbar_blocks, nullptr, (cudaStream_t)stream));
 }
 
 qsa_status_t qsa_index_score_topk(const qsa_config_t *cfg, const void *qi, const float *kbar,

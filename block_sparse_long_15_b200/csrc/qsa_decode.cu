@@ -18,8 +18,6 @@
 #include <math.h>
 #include <stdio.h>
 
-#include <mutex>
-
 #include "qsa_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -856,31 +854,11 @@ cudaError_t launch_attn_decode(const Dims &D, const Seqs &S, const void *q, cons
 // ---------------------------------------------------------------------------
 namespace {
 
-// Split partials of qsa_sparse_attn_decode_noalloc: every GPU that loads the
-// library holds this array until the process exits.
+// Status word and split partials of qsa_sparse_attn_decode_noalloc: every GPU that
+// loads the library holds this array until the process exits. Layout: [0, 256) the
+// status word the decode kernels record a timed-out wait in, then the decode
+// workspace (unit counters, then the partials).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[QSA_NOALLOC_SCRATCH_BYTES];
-
-std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[256];  // device address of the array, per device ordinal
-
-// Device address of the array on the current device. The array's name is only a
-// host-side stand-in in host code; its device address comes from
-// cudaGetSymbolAddress, called once per device with that device current.
-cudaError_t noalloc_scratch(void **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
-  return cudaSuccess;
-}
 
 }  // namespace
 
@@ -908,7 +886,7 @@ extern "C" qsa_status_t qsa_sparse_attn_decode_noalloc(const qsa_config_t *cfg, 
   S.n_q = 1;
   S.kv_cap = kv_cap;
   S.nb_cap = kv_cap / D.B;
-  const size_t need = attn_decode_workspace(D, S);
+  const size_t need = kStatusBytes + attn_decode_workspace(D, S);
   if (need > (size_t)QSA_NOALLOC_SCRATCH_BYTES) {
     char what[160];
     snprintf(what, sizeof what, "decode partials need %zu bytes, more than the %d-byte static scratch", need,
@@ -916,19 +894,29 @@ extern "C" qsa_status_t qsa_sparse_attn_decode_noalloc(const qsa_config_t *cfg, 
     note_error(what, cudaErrorInvalidValue);
     return QSA_ERR_UNSUPPORTED;
   }
-  void *scratch = nullptr;
-  cudaError_t e = noalloc_scratch(&scratch);
+  // In host code the array's name only stands in for it; its device address on the
+  // current device comes from the runtime. The lookup is made on every call (a
+  // host-side table lookup once the module is loaded), so that an address is never
+  // reused after the device's context was torn down and the module loaded again.
+  void *arr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&arr, g_noalloc_scratch);
   if (e != cudaSuccess) {
     note_error("cudaGetSymbolAddress of the static decode scratch", e);
     return QSA_ERR_CUDA;
   }
-  // No device-side status word here (it would need a caller buffer or a sync to
-  // read): lengths that do not fit the cache are skipped without a report.
-  e = launch_attn_decode(D, S, q, k, v, sel, out, scratch, need, nullptr, (cudaStream_t)stream);
+  // Clear the status word and the unit counters, ordered before the kernel on the
+  // stream: a call whose bounded wait ran out leaves counters set, and this keeps
+  // that from reaching any later call.
+  e = cudaMemsetAsync(arr, 0, kStatusBytes + counters_bytes(D, S), (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    note_error("qsa_sparse_attn_decode_noalloc: clearing the static scratch", e);
+    return QSA_ERR_CUDA;
+  }
+  e = launch_attn_decode(D, S, q, k, v, sel, out, (char *)arr + kStatusBytes, need - kStatusBytes, (int *)arr,
+                         (cudaStream_t)stream);
   if (e != cudaSuccess) {
     note_error("qsa_sparse_attn_decode_noalloc launch", e);
     return e == cudaErrorNotSupported ? QSA_ERR_UNSUPPORTED : QSA_ERR_CUDA;
   }
   return QSA_OK;
 }
-

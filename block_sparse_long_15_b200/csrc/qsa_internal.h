@@ -92,8 +92,20 @@ cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi,
 // holds the hi/lo planes (score_tc_workspace bytes).
 bool score_tc_supported(const Dims &D, const Seqs &S);
 size_t score_tc_workspace(const Dims &D, const Seqs &S);
+// With scores_out set, writes each row's scores s[b][r][j] (j < n_c of the row) to
+// scores_out [batch][n_q][nb_cap] instead of selecting (sel is not touched).
 cudaError_t launch_score_topk_tc(const Dims &D, const Seqs &S, const void *qi, const float *kbar, int32_t *sel,
-                                 void *scratch, int *status, cudaStream_t st);
+                                 void *scratch, int *status, cudaStream_t st, float *scores_out = nullptr);
+
+// Steps 2 alone on CUDA cores (fp32): each row's scores s[b][r][j], j < n_c, into
+// scores [batch][n_q][nb_cap]; other entries are not written.
+cudaError_t launch_index_scores_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
+                                     float *scores, int *status, cudaStream_t st);
+
+// Step 3 alone: top-k of each row of a score matrix [batch][n_q][nb_cap] (any finite
+// fp32 values, e.g. the sum of head-sharded partial scores), ties to the lower block.
+cudaError_t launch_select_topk(const Dims &D, const Seqs &S, const float *scores, int32_t *sel, int *status,
+                               cudaStream_t st);
 
 // The decode prologue (append the new token at kv_len - 1, compress a block it
 // completes, advance kbar_blocks; see launch_decode_append) fused with steps 2+3

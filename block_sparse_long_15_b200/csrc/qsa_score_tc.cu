@@ -38,6 +38,7 @@ struct ScoreParams {
   Dims D;
   Seqs S;
   int32_t *sel;
+  float *scores_out;  // if set: write the rows' scores [batch][n_q][nb_cap] here, select nothing
   int *status;
   int n_tiles;  // token tiles per sequence
   int N;        // kTok * Hi
@@ -58,6 +59,133 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
+}
+
+// Exact top-k of one row by a warp: writes out[0 .. k) with the ids of the k largest
+// keys in ascending id order, ties to the lower id, -1 padded; n < 0 marks a padding
+// row (all -1) and n <= k keeps every id. key(j) returns the 32-bit key of id j whose
+// unsigned order is the score order (fp32 bit patterns of scores >= +0, or the
+// order-preserving map of any finite fp32). wh: 256 ints of shared memory for the warp.
+//
+// The k-th largest key is found by 8-bit radix passes from the highest bit in which
+// the row's keys differ (the bits above it are common to all keys, so no pass piles
+// every key into one bin); once the keys still matching the prefix are at most 32,
+// they are gathered one per lane and sorted across the warp (bitonic, descending),
+// which settles the k-th key and how many ties of it to keep. Then keys above it,
+// and the lowest-id keys equal to it, are written in id order.
+template <typename KeyFn>
+__device__ __forceinline__ void warp_select_row(KeyFn key_of, int n, int k, int32_t *out, int *wh) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = lanemask_lt();
+  if (n <= k) {  // padding row (n = -1), or every complete block kept
+    for (int i = lane; i < k; i += 32) out[i] = (i < n) ? i : -1;
+    return;
+  }
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int j = lane; j < n; j += 32) {
+    const uint32_t key = key_of(j);
+    kmin = min(kmin, key);
+    kmax = max(kmax, key);
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  const uint32_t diff = kmin ^ kmax;
+  const int top = diff ? 31 - __clz(diff) : -1;
+  uint32_t pmask = top >= 31 ? 0u : (0xffffffffu << (top + 1));
+  uint32_t prefix = kmax & pmask;
+  int remaining = k;
+  auto settle = [&]() {
+    __syncwarp();
+    int base = 0;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < n ? key_of(j) : 0u;
+      const bool cand = j < n && (key & pmask) == prefix;
+      const unsigned m = __ballot_sync(0xffffffffu, cand);
+      if (cand) wh[base + __popc(m & lt)] = (int)key;
+      base += __popc(m);
+    }
+    __syncwarp();
+    uint32_t v = lane < base ? (uint32_t)wh[lane] : 0u;
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const uint32_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+        // descending runs where (lane & size) == 0, ascending otherwise; the last
+        // merge (size 32) leaves the whole warp descending
+        const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
+        v = keep_max ? max(v, o) : min(v, o);
+      }
+    }
+    const uint32_t val = __shfl_sync(0xffffffffu, v, remaining - 1);
+    remaining -= __popc(__ballot_sync(0xffffffffu, lane < base && v > val));
+    prefix = val;
+    pmask = 0xffffffffu;
+    __syncwarp();
+  };
+  if (top >= 0 && n <= 32) settle();
+  for (int hi_bit = top; hi_bit >= 0 && pmask != 0xffffffffu; hi_bit -= 8) {
+    const int shift = hi_bit >= 7 ? hi_bit - 7 : 0;
+    const uint32_t dmask = (2u << (hi_bit - shift)) - 1u;
+    for (int i = lane; i < 256; i += 32) wh[i] = 0;
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const uint32_t key = key_of(j);
+      if ((key & pmask) == prefix) atomicAdd(&wh[(key >> shift) & dmask], 1);
+    }
+    __syncwarp();
+    // lane L owns digits 255-8L .. 248-8L (descending)
+    int c[8], tot = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      c[q] = wh[255 - 8 * lane - q];
+      tot += c[q];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int excl = incl - tot;
+    int digit = 0, above = 0, cnt = 0;
+    const bool mine = excl < remaining && incl >= remaining;
+    if (mine) {
+      above = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (above + c[q] >= remaining) {
+          digit = 255 - 8 * lane - q;
+          cnt = c[q];
+          break;
+        }
+        above += c[q];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    cnt = __shfl_sync(0xffffffffu, cnt, src);
+    prefix |= (uint32_t)digit << shift;
+    pmask |= dmask << shift;
+    remaining -= above;
+    __syncwarp();
+    if (shift > 0 && cnt <= 32) settle();
+  }
+  int base_i = 0, tie_base = 0;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < n ? key_of(j) : 0u;
+    const bool gt = j < n && key > prefix;
+    const bool eq = j < n && key == prefix;
+    const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && tie_base + __popc(eq_mask & lt) < remaining);
+    const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+    if (take) out[base_i + __popc(take_mask & lt)] = j;
+    base_i += __popc(take_mask);
+    tie_base += __popc(eq_mask);
+  }
 }
 
 template <int HI>
@@ -183,7 +311,10 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
             const float x = __uint_as_float(v[tq * Hi + h]);
             s += x > 0.f ? x : 0.f;
           }
-          if (j < ncs[tok]) scores[tok * row_stride + j] = __float_as_uint(s);
+          if (j < ncs[tok]) {
+            if (P.scores_out) P.scores_out[((size_t)b * S.n_q + r0 + tok) * S.nb_cap + j] = s;
+            else scores[tok * row_stride + j] = __float_as_uint(s);
+          }
         }
       }
       tc_fence_before();
@@ -200,130 +331,41 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
   }
 
   // ---------------------------------------------------------------- per-token top-k
+  if (P.scores_out) return;  // partial scores only: the caller reduces and selects
   int *wh = hist + warp * 256;
-  const unsigned lt = lanemask_lt();
   for (int tok = warp; tok < kTok; tok += kThreads / 32) {
     const int r = r0 + tok;
     if (r >= S.n_q) continue;
-    int32_t *out = P.sel + ((size_t)b * S.n_q + r) * D.k;
-    const int n = ncs[tok];
-    if (n <= D.k) {  // padding row (n = -1), or every complete block kept
-      for (int i = lane; i < D.k; i += 32) out[i] = (i < n) ? i : -1;
-      continue;
-    }
     const uint32_t *keys = scores + tok * row_stride;
-    // Bits above the highest one in which the row's keys differ are common to all
-    // keys: the radix passes start below them, 8 bits at a time, so that no pass
-    // piles every key into one histogram bin.
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int j = lane; j < n; j += 32) {
-      kmin = min(kmin, keys[j]);
-      kmax = max(kmax, keys[j]);
-    }
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    const uint32_t diff = kmin ^ kmax;
-    const int top = diff ? 31 - __clz(diff) : -1;
-    uint32_t pmask = top >= 31 ? 0u : (0xffffffffu << (top + 1));
-    uint32_t prefix = kmax & pmask;
-    int remaining = D.k;
-    // Once the keys still matching the prefix are at most 32, the rest is settled in
-    // registers: they are gathered one per lane, sorted descending (bitonic, across
-    // the warp), and the remaining-th of them is the k-th largest key; the keys above
-    // it among them leave `remaining` ties to take.
-    auto settle = [&]() {
-      __syncwarp();
-      int base = 0;
-      for (int j0 = 0; j0 < n; j0 += 32) {
-        const int j = j0 + lane;
-        const uint32_t key = j < n ? keys[j] : 0u;
-        const bool cand = j < n && (key & pmask) == prefix;
-        const unsigned m = __ballot_sync(0xffffffffu, cand);
-        if (cand) wh[base + __popc(m & lt)] = (int)key;
-        base += __popc(m);
-      }
-      __syncwarp();
-      uint32_t v = lane < base ? (uint32_t)wh[lane] : 0u;
-#pragma unroll
-      for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          const uint32_t o = __shfl_xor_sync(0xffffffffu, v, stride);
-          // descending runs where (lane & size) == 0, ascending otherwise; the last
-          // merge (size 32) leaves the whole warp descending
-          const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
-          v = keep_max ? max(v, o) : min(v, o);
-        }
-      }
-      const uint32_t val = __shfl_sync(0xffffffffu, v, remaining - 1);
-      remaining -= __popc(__ballot_sync(0xffffffffu, lane < base && v > val));
-      prefix = val;
-      pmask = 0xffffffffu;
-      __syncwarp();
-    };
-    if (top >= 0 && n <= 32) settle();
-    for (int hi_bit = top; hi_bit >= 0 && pmask != 0xffffffffu; hi_bit -= 8) {
-      const int shift = hi_bit >= 7 ? hi_bit - 7 : 0;
-      const uint32_t dmask = (2u << (hi_bit - shift)) - 1u;
-      for (int i = lane; i < 256; i += 32) wh[i] = 0;
-      __syncwarp();
-      for (int j = lane; j < n; j += 32) {
-        const uint32_t key = keys[j];
-        if ((key & pmask) == prefix) atomicAdd(&wh[(key >> shift) & dmask], 1);
-      }
-      __syncwarp();
-      // lane L owns digits 255-8L .. 248-8L (descending)
-      int c[8], tot = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        c[q] = wh[255 - 8 * lane - q];
-        tot += c[q];
-      }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const int excl = incl - tot;
-      int digit = 0, above = 0, cnt = 0;
-      const bool mine = excl < remaining && incl >= remaining;
-      if (mine) {
-        above = excl;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (above + c[q] >= remaining) {
-            digit = 255 - 8 * lane - q;
-            cnt = c[q];
-            break;
-          }
-          above += c[q];
-        }
-      }
-      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      above = __shfl_sync(0xffffffffu, above, src);
-      cnt = __shfl_sync(0xffffffffu, cnt, src);
-      prefix |= (uint32_t)digit << shift;
-      pmask |= dmask << shift;
-      remaining -= above;
-      __syncwarp();
-      if (shift > 0 && cnt <= 32) settle();
-    }
-    int base_i = 0, tie_base = 0;
-    for (int j0 = 0; j0 < n; j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t key = j < n ? keys[j] : 0u;
-      const bool gt = j < n && key > prefix;
-      const bool eq = j < n && key == prefix;
-      const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
-      const bool take = gt || (eq && tie_base + __popc(eq_mask & lt) < remaining);
-      const unsigned take_mask = __ballot_sync(0xffffffffu, take);
-      if (take) out[base_i + __popc(take_mask & lt)] = j;
-      base_i += __popc(take_mask);
-      tie_base += __popc(eq_mask);
-    }
+    warp_select_row([&](int j) { return keys[j]; }, ncs[tok], D.k, P.sel + ((size_t)b * S.n_q + r) * D.k, wh);
   }
+}
+
+// Step 3 from a score matrix: one warp per query row reads the row's n_c candidate
+// scores from scores [batch][n_q][nb_cap] (through the order-preserving map of fp32
+// to uint32, so any finite value orders correctly; -0 counts as +0) and selects as
+// the fused kernels do.
+constexpr int kSelWarps = 8;
+__global__ void __launch_bounds__(kSelWarps * 32)
+k_select_topk(Dims D, Seqs S, const float *__restrict__ scores, int32_t *__restrict__ sel, int *status) {
+  __shared__ int hist[kSelWarps][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kSelWarps + warp;  // over batch * n_q
+  if (row >= (long long)S.batch * S.n_q) return;
+  const int b = (int)(row / S.n_q), r = (int)(row % S.n_q);
+  const bool ok = seq_ok(S, b, lane == 0 ? status : nullptr);
+  const int len = ok ? S.kv_len[b] : 0;
+  const int t = seq_qfirst(S, b) + r;
+  const int n = (ok && t >= 0 && t < len) ? (t + 1) / D.B : -1;
+  const float *srow = scores + (size_t)row * S.nb_cap;
+  warp_select_row(
+      [&](int j) {
+        float f = __ldg(srow + j);
+        if (f == 0.f) f = 0.f;
+        const uint32_t u = __float_as_uint(f);
+        return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+      },
+      n, D.k, sel + (size_t)row * D.k, hist[warp]);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -383,7 +425,7 @@ size_t score_tc_workspace(const Dims &D, const Seqs &S) {
 }
 
 cudaError_t launch_score_topk_tc(const Dims &D, const Seqs &S, const void *qi, const float *kbar, int32_t *sel,
-                                 void *scratch, int *status, cudaStream_t st) {
+                                 void *scratch, int *status, cudaStream_t st, float *scores_out) {
   if (S.batch == 0 || S.n_q == 0) return cudaSuccess;
   const size_t plane = ((size_t)S.batch * S.nb_cap * D.di * 2 + 255) & ~(size_t)255;
   __nv_bfloat16 *hi = (__nv_bfloat16 *)scratch;
@@ -404,6 +446,7 @@ cudaError_t launch_score_topk_tc(const Dims &D, const Seqs &S, const void *qi, c
   P.D = D;
   P.S = S;
   P.sel = sel;
+  P.scores_out = scores_out;
   P.status = status;
   P.n_tiles = (S.n_q + kTok - 1) / kTok;
   P.N = kTok * D.Hi;
@@ -415,6 +458,17 @@ cudaError_t launch_score_topk_tc(const Dims &D, const Seqs &S, const void *qi, c
   if (e != cudaSuccess) return e;
   note_launch();
   kern<<<dim3(P.n_tiles, S.batch), kThreads, smem, st>>>(tq, th, tl, P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_topk(const Dims &D, const Seqs &S, const float *scores, int32_t *sel, int *status,
+                               cudaStream_t st) {
+  const long long rows = (long long)S.batch * S.n_q;
+  if (rows == 0) return cudaSuccess;
+  const long long grid = (rows + kSelWarps - 1) / kSelWarps;
+  if (grid > 0x7fffffffLL) return cudaErrorNotSupported;
+  note_launch();
+  k_select_topk<<<(unsigned)grid, kSelWarps * 32, 0, st>>>(D, S, scores, sel, status);
   return cudaGetLastError();
 }
 

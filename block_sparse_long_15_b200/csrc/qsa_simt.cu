@@ -99,7 +99,7 @@ k_compress(Dims D, Seqs S, const T *__restrict__ ki, const int32_t *__restrict__
 template <typename T>
 __global__ void k_score_topk_simt(Dims D, Seqs S, const T *__restrict__ qi,
                                   const float *__restrict__ kbar, int32_t *__restrict__ sel,
-                                  int *status, int warps, int nc_cap) {
+                                  int *status, int warps, int nc_cap, float *__restrict__ scores_out) {
   extern __shared__ float smem[];
   const int HD = D.Hi * D.di;
   float *qi_s = smem;                                  // [warps][Hi*di]
@@ -145,10 +145,11 @@ __global__ void k_score_topk_simt(Dims D, Seqs S, const T *__restrict__ qi,
         s += dot > 0.f ? dot : 0.f;
       }
       keys[j] = __float_as_uint(s);
+      if (scores_out) scores_out[((size_t)b * S.n_q + r) * S.nb_cap + j] = s;
     }
   }
   __syncwarp();
-  if (r >= S.n_q) return;
+  if (r >= S.n_q || scores_out) return;  // with scores_out: scores only, no selection
   int32_t *out = sel + ((size_t)b * S.n_q + r) * D.k;
   if (!valid || n_c <= D.k) {
     for (int i = lane; i < D.k; i += 32) out[i] = (i < n_c) ? i : -1;
@@ -662,10 +663,12 @@ static size_t score_smem(const Dims &D, int warps, int nc_cap) {
   return sizeof(float) * ((size_t)warps * D.Hi * D.di + 32 * (D.di + 1) + (size_t)warps * nc_cap);
 }
 
-cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
-                                   int32_t *sel, int *status, cudaStream_t st) {
+// With scores_out set: the warp-per-row kernel writes each row's scores there and
+// selects nothing (the CTA-per-row kernel is not used).
+static cudaError_t launch_score_topk_simt_impl(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
+                                               int32_t *sel, int *status, cudaStream_t st, float *scores_out) {
   if (S.batch == 0 || S.n_q == 0) return cudaSuccess;
-  if ((long long)S.batch * S.n_q <= 4096 && D.di % 4 == 0) {
+  if (!scores_out && (long long)S.batch * S.n_q <= 4096 && D.di % 4 == 0) {
     // few rows: one CTA per row
     const size_t smem = sizeof(float) * ((size_t)D.Hi * D.di + D.di + S.nb_cap);
     if (smem <= 200 * 1024) {
@@ -697,14 +700,25 @@ cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi,
     auto kern = k_score_topk_simt<__nv_bfloat16>;
     e = ensure_smem(kern, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, warps * 32, smem, st>>>(D, S, (const __nv_bfloat16 *)qi, kbar, sel, status, warps, nc_cap);
+    kern<<<grid, warps * 32, smem, st>>>(D, S, (const __nv_bfloat16 *)qi, kbar, sel, status, warps, nc_cap,
+                                         scores_out);
   } else {
     auto kern = k_score_topk_simt<float>;
     e = ensure_smem(kern, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, warps * 32, smem, st>>>(D, S, (const float *)qi, kbar, sel, status, warps, nc_cap);
+    kern<<<grid, warps * 32, smem, st>>>(D, S, (const float *)qi, kbar, sel, status, warps, nc_cap, scores_out);
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_index_scores_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
+                                     float *scores, int *status, cudaStream_t st) {
+  return launch_score_topk_simt_impl(D, S, qi, kbar, nullptr, status, st, scores);
+}
+
+cudaError_t launch_score_topk_simt(const Dims &D, const Seqs &S, const void *qi, const float *kbar,
+                                   int32_t *sel, int *status, cudaStream_t st) {
+  return launch_score_topk_simt_impl(D, S, qi, kbar, sel, status, st, nullptr);
 }
 
 cudaError_t launch_decode_append_score(const Dims &D, const Seqs &S, const DecodeAppend &A, const void *qi,

@@ -59,7 +59,7 @@ def _load() -> ctypes.CDLL:
         "qsa_topk_blocks": ([cfgp], I),
         "qsa_status_string": ([I], ctypes.c_char_p),
         "qsa_workspace_size": ([cfgp, I, I, I, I, P(S)], I),
-        "qsa_compress_blocks": ([cfgp, V, V, V, V, I, I, V, V], I),
+        "qsa_compress_blocks": ([cfgp, V, V, V, V, I, I, V, V, V], I),
         "qsa_index_score_topk": ([cfgp, V, V, V, V, I, I, I, V, V, S, V], I),
         "qsa_sparse_attn": ([cfgp, V, V, V, V, V, V, V, I, I, I, V, V, S, V], I),
         "qsa_forward": ([cfgp, I, P(qsa_tensors_t), V, S, V], I),
@@ -144,6 +144,14 @@ def _want(t: torch.Tensor, dtype: torch.dtype, shape, name: str):
         raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _want_lengths(batch: int, **named):
+    """Per-sequence int32 vectors of `batch` entries (kv_start, kv_len, q_first, ...)."""
+    for name, t in named.items():
+        if t is None:
+            raise ValueError(f"{name}: required")
+        _want(t, torch.int32, (batch,), name)
+
+
 # --------------------------------------------------------------------------- entry points
 def qsa_config_validate(cfg: qsa_config_t) -> int:
     return _lib.qsa_config_validate(ctypes.byref(cfg))
@@ -183,18 +191,27 @@ def alloc_workspace(cfg: qsa_config_t, mode: int, batch: int, n_q: int, kv_cap: 
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
-def qsa_compress_blocks(cfg, ki, kv_start, kv_len, kbar, blocks_done=None, stream=None):
+def qsa_compress_blocks(cfg, ki, kv_start, kv_len, kbar, blocks_done=None, kbar_blocks=None, stream=None):
+    """k̄ of the complete blocks; kbar_blocks (optional, int32 [batch]) receives kv_len // B."""
     batch, kv_cap = ki.shape[0], ki.shape[1]
     _want(ki, _elem(cfg), (batch, kv_cap, cfg.indexer_head_dim), "ki")
     _want(kbar, torch.float32, (batch, kv_cap // cfg.indexer_compress_ratio, cfg.indexer_head_dim), "kbar")
+    _want_lengths(batch, kv_start=kv_start, kv_len=kv_len)
+    if blocks_done is not None:
+        _want_lengths(batch, blocks_done=blocks_done)
+    if kbar_blocks is not None:
+        _want_lengths(batch, kbar_blocks=kbar_blocks)
     _check(_lib.qsa_compress_blocks(ctypes.byref(cfg), _p(ki), _p(kv_start), _p(kv_len), _p(blocks_done),
-                                    batch, kv_cap, _p(kbar), _stream(stream)), "qsa_compress_blocks")
+                                    batch, kv_cap, _p(kbar), _p(kbar_blocks), _stream(stream)),
+           "qsa_compress_blocks")
 
 
 def qsa_index_score_topk(cfg, qi, kbar, kv_len, q_first, kv_cap, sel, workspace, stream=None):
     batch, n_q = qi.shape[0], qi.shape[1]
     _want(qi, _elem(cfg), (batch, n_q, cfg.indexer_n_heads, cfg.indexer_head_dim), "qi")
     _want(sel, torch.int32, (batch, n_q, qsa_topk_blocks(cfg)), "sel")
+    _want(kbar, torch.float32, (batch, kv_cap // cfg.indexer_compress_ratio, cfg.indexer_head_dim), "kbar")
+    _want_lengths(batch, kv_len=kv_len, q_first=q_first)
     _check(_lib.qsa_index_score_topk(ctypes.byref(cfg), _p(qi), _p(kbar), _p(kv_len), _p(q_first), batch,
                                      n_q, kv_cap, _p(sel), _p(workspace), workspace.numel(),
                                      _stream(stream)), "qsa_index_score_topk")
@@ -208,6 +225,8 @@ def qsa_sparse_attn(cfg, q, k, v, sel, kv_start, kv_len, q_first, out, workspace
     _want(k, dt, (batch, cfg.num_key_value_heads, kv_cap, cfg.head_dim), "k")
     _want(v, dt, (batch, cfg.num_key_value_heads, kv_cap, cfg.head_dim), "v")
     _want(out, dt, (batch, n_q, cfg.num_attention_heads, cfg.head_dim), "out")
+    _want(sel, torch.int32, (batch, n_q, qsa_topk_blocks(cfg)), "sel")
+    _want_lengths(batch, kv_start=kv_start, kv_len=kv_len, q_first=q_first)
     _check(_lib.qsa_sparse_attn(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(kv_start), _p(kv_len),
                                 _p(q_first), batch, n_q, kv_cap, _p(out), _p(workspace),
                                 workspace.numel(), _stream(stream)), "qsa_sparse_attn")
@@ -241,6 +260,10 @@ def qsa_sparse_attn_decode_noalloc(cfg, q, k, v, sel, kv_start, kv_len, out, str
     kv_cap = k.shape[2]
     dt = _elem(cfg)
     _want(q, dt, (batch, 1, cfg.num_attention_heads, cfg.head_dim), "q")
+    _want(k, dt, (batch, cfg.num_key_value_heads, kv_cap, cfg.head_dim), "k")
+    _want(v, dt, (batch, cfg.num_key_value_heads, kv_cap, cfg.head_dim), "v")
+    _want(sel, torch.int32, (batch, 1, qsa_topk_blocks(cfg)), "sel")
+    _want_lengths(batch, kv_start=kv_start, kv_len=kv_len)
     _want(out, dt, (batch, 1, cfg.num_attention_heads, cfg.head_dim), "out")
     _check(_lib.qsa_sparse_attn_decode_noalloc(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(kv_start),
                                                _p(kv_len), batch, kv_cap, _p(out), _stream(stream)),

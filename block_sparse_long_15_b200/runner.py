@@ -17,22 +17,60 @@ def to_device(inp: Dict[str, torch.Tensor], device="cuda") -> Dict[str, torch.Te
     return {k: v.to(device, non_blocking=True).contiguous() for k, v in inp.items()}
 
 
+GUARD_BYTES = 4096          # guard band on each side of a guarded output buffer
+GUARD_WORD = 0x5A5A5A5A      # the pattern the bands are filled with, as int32 words
+
+
+class Guarded:
+    """A contiguous output tensor with a guard band of GUARD_BYTES on each side, filled
+    with GUARD_WORD. `view` is the tensor handed to the library (256-byte aligned);
+    intact() tells whether a call wrote outside it."""
+
+    def __init__(self, shape, dtype, device="cuda"):
+        n = 1
+        for x in shape:
+            n *= int(x)
+        esz = torch.empty((), dtype=dtype).element_size()
+        body = (n * esz + 255) // 256 * 256
+        self.raw = torch.empty(2 * GUARD_BYTES + body, dtype=torch.uint8, device=device)
+        self.raw.view(torch.int32).fill_(GUARD_WORD)
+        self.body = body
+        self.view = self.raw[GUARD_BYTES:GUARD_BYTES + n * esz].view(dtype).view(*shape)
+
+    def intact(self) -> bool:
+        lo = self.raw[:GUARD_BYTES].view(torch.int32)
+        hi = self.raw[GUARD_BYTES + self.body:].view(torch.int32)
+        want = GUARD_WORD
+        return bool((lo == want).all().item()) and bool((hi == want).all().item())
+
+
+def _outputs(shape_out, dtype, shape_sel, device, guard: bool):
+    if not guard:
+        return (torch.empty(shape_out, dtype=dtype, device=device),
+                torch.empty(shape_sel, dtype=torch.int32, device=device), [])
+    go, gs = Guarded(shape_out, dtype, device), Guarded(shape_sel, torch.int32, device)
+    return go.view, gs.view, [go, gs]
+
+
 class QSAPrefill:
     """One prefill call: compress every complete block, score, select, attend."""
 
-    def __init__(self, w, inp: Dict[str, torch.Tensor], device="cuda"):
+    def __init__(self, w, inp: Dict[str, torch.Tensor], device="cuda", guard: bool = False):
         self.cfg = qsa.config_for(w)
         self.k = qsa.qsa_topk_blocks(self.cfg)
         g = to_device(inp, device)
         B, n_q = g["q"].shape[0], g["q"].shape[1]
         kv_cap = g["k"].shape[2]
+        out, sel, self.guards = _outputs(g["q"].shape, g["q"].dtype, (B, n_q, self.k), device, guard)
         self.t = dict(q=g["q"], qi=g["qi"], k_cache=g["k"], v_cache=g["v"], ki_cache=g["ki"],
                       kbar_cache=torch.zeros(B, kv_cap // w.block, w.di, dtype=torch.float32, device=device),
                       kbar_blocks=torch.zeros(B, dtype=torch.int32, device=device),
-                      kv_start=g["kv_start"], kv_len=g["kv_len"], q_first=g["q_first"],
-                      sel=torch.empty(B, n_q, self.k, dtype=torch.int32, device=device),
-                      out=torch.empty_like(g["q"]))
+                      kv_start=g["kv_start"], kv_len=g["kv_len"], q_first=g["q_first"], sel=sel, out=out)
         self.ws = qsa.alloc_workspace(self.cfg, qsa.QSA_PREFILL, B, n_q, kv_cap, device)
+
+    def guards_intact(self) -> bool:
+        """With guard=True: no call wrote past either end of `out` or `sel`."""
+        return all(x.intact() for x in self.guards)
 
     def __call__(self, stream=None):
         qsa.qsa_forward(self.cfg, qsa.QSA_PREFILL, self.t, self.ws, stream)
@@ -51,29 +89,30 @@ class QSADecode:
     steady-state step) -- reset_state() rewinds kbar_blocks for that.
     """
 
-    def __init__(self, w, inp: Dict[str, torch.Tensor], device="cuda"):
+    def __init__(self, w, inp: Dict[str, torch.Tensor], device="cuda", guard: bool = False):
         self.cfg = qsa.config_for(w)
         self.k = qsa.qsa_topk_blocks(self.cfg)
         self.w = w
         g = to_device(inp, device)
         B = g["q"].shape[0]
         kv_cap = g["k"].shape[2]
+        out, sel, self.guards = _outputs(g["q"].shape, g["q"].dtype, (B, 1, self.k), device, guard)
         self.t = dict(q=g["q"], qi=g["qi"], k_cache=g["k"], v_cache=g["v"], ki_cache=g["ki"],
                       kbar_cache=torch.zeros(B, kv_cap // w.block, w.di, dtype=torch.float32, device=device),
                       kbar_blocks=torch.zeros(B, dtype=torch.int32, device=device),
                       k_new=g["k_new"], v_new=g["v_new"], ki_new=g["ki_new"],
-                      kv_start=g["kv_start"], kv_len=g["kv_len"],
-                      sel=torch.empty(B, 1, self.k, dtype=torch.int32, device=device),
-                      out=torch.empty_like(g["q"]))
+                      kv_start=g["kv_start"], kv_len=g["kv_len"], sel=sel, out=out)
         self.prev_len = (g["kv_len"] - 1).contiguous()
-        # indexer state for the tokens already cached: blocks [0, (L-1)/B)
+        # indexer state for the tokens already cached: k̄ of blocks [0, (L-1)/B) and
+        # their count, both written by the library
         qsa.qsa_compress_blocks(self.cfg, self.t["ki_cache"], self.t["kv_start"], self.prev_len,
-                                self.t["kbar_cache"])
+                                self.t["kbar_cache"], kbar_blocks=self.t["kbar_blocks"])
+        self._blocks0 = self.t["kbar_blocks"].clone()
         self.ws = qsa.alloc_workspace(self.cfg, qsa.QSA_DECODE, B, 1, kv_cap, device)
-        self.reset_state()
 
     def reset_state(self):
-        self.t["kbar_blocks"].copy_(torch.div(self.prev_len, self.w.block, rounding_mode="floor"))
+        """Rewind the indexer state's block count to what it was before the first step."""
+        self.t["kbar_blocks"].copy_(self._blocks0)
 
     def __call__(self, stream=None):
         qsa.qsa_forward(self.cfg, qsa.QSA_DECODE, self.t, self.ws, stream)
@@ -81,6 +120,10 @@ class QSADecode:
 
     def status(self) -> int:
         return qsa.qsa_read_device_status(self.ws)
+
+    def guards_intact(self) -> bool:
+        """With guard=True: no call wrote past either end of `out` or `sel`."""
+        return all(x.intact() for x in self.guards)
 
 
 class QSADecodeOffload(QSADecode):

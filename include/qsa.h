@@ -66,7 +66,7 @@
 extern "C" {
 #endif
 
-#define QSA_ABI_VERSION 1
+#define QSA_ABI_VERSION 2
 
 typedef struct CUstream_st *qsa_stream_t; /* same type as cudaStream_t */
 
@@ -128,8 +128,9 @@ const char *qsa_status_string(qsa_status_t status);
 /* Bytes of workspace the calls below need for these sizes (mode QSA_PREFILL or
  * QSA_DECODE). The workspace is caller-owned device memory, 256-byte aligned, and
  * must be all zero before its first use; the library leaves the parts it relies on
- * at zero again after each call. Its first 256 bytes hold the status word
- * (qsa_read_device_status reads and clears it). One workspace must not serve two
+ * at zero again after each call, except after a call whose device wait ran out
+ * (status QSA_ERR_TIMEOUT): zero the workspace again before reusing it. Its first
+ * 256 bytes hold the status word (qsa_read_device_status reads and clears it). One workspace must not serve two
  * calls that run concurrently. */
 qsa_status_t qsa_workspace_size(const qsa_config_t *cfg, int32_t mode, int32_t batch, int32_t n_q,
                                 int32_t kv_cap, size_t *bytes);
@@ -137,10 +138,13 @@ qsa_status_t qsa_workspace_size(const qsa_config_t *cfg, int32_t mode, int32_t b
 /* Step 1, block compression (Qwen4ExpTextConfig indexer_compress_ratio: B consecutive
  * indexer keys averaged into one block). For each sequence writes kbar[b][j] for the
  * complete blocks blocks_done[b] <= j < kv_len[b] / B (blocks_done may be NULL: all
- * complete blocks). fp32 sum in key order, then divided by B. */
+ * complete blocks). fp32 sum in key order, then divided by B. kbar_blocks (may be
+ * NULL) receives kv_len[b] / B, the count of compressed blocks the indexer state
+ * then holds -- what a decode step expects in qsa_tensors_t.kbar_blocks when the
+ * cache holds kv_len[b] tokens. */
 qsa_status_t qsa_compress_blocks(const qsa_config_t *cfg, const void *ki, const int32_t *kv_start,
                                  const int32_t *kv_len, const int32_t *blocks_done, int32_t batch,
-                                 int32_t kv_cap, float *kbar, qsa_stream_t stream);
+                                 int32_t kv_cap, float *kbar, int32_t *kbar_blocks, qsa_stream_t stream);
 
 /* Steps 2 and 3, scoring and causal top-k selection (intro paragraph: multiple query
  * heads score compressed key blocks, the most relevant blocks are selected;
@@ -210,22 +214,26 @@ qsa_status_t qsa_selftest_wait_timeout(void *workspace, int64_t limit_ns, qsa_st
  * input and output buffers, or a serving process that reserves all device memory
  * for its own pool, so that a cudaMalloc would fail or go around that pool. It
  * computes what qsa_sparse_attn computes for n_q == 1 with q_first[b] = kv_len[b] - 1,
- * and allocates nothing: the split partials of the decode kernel live in a fixed
- * array of QSA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
- * the library holds until the process exits (the paper has no counterpart; this is
- * an interface convenience).
+ * and allocates nothing: a status word and the split partials of the decode kernel
+ * live in a fixed array of QSA_NOALLOC_SCRATCH_BYTES inside the library, which every
+ * GPU that loads the library holds until the process exits (the paper has no
+ * counterpart; this is an interface convenience).
  *   Arguments and layouts as for qsa_sparse_attn with n_q = 1 (q, out [batch][1][Hq][d];
  *   k, v [batch][Hkv][kv_cap][d]; sel [batch][1][k]); bf16, head_dim 128, B = 64, G <= 8.
- *   The first call on a device looks up the array's device address (with that device
- *   current); make that first call before any stream capture.
- *   Every call on a device shares the one array and leaves its partials there; calls
- *   that overlap on the GPU (e.g. on two streams) race on it and must be serialised
- *   by the caller.
+ *   Each call looks up the array's device address on the current device (a host-side
+ *   lookup; the first one on a device may load the library's device code, so make
+ *   that first call before any stream capture), then enqueues on `stream` a clear of
+ *   the array's status word and unit counters followed by the kernel: a call never
+ *   sees what an earlier one left there.
+ *   Every call on a device shares the one array; calls that overlap on the GPU (e.g.
+ *   on two streams) race on it and must be serialised by the caller.
  *   Returns QSA_ERR_UNSUPPORTED (and sets qsa_last_error) when the partials of this
  *   batch exceed the array -- with batch * Hkv <= 2048 they take about
  *   (batch * Hkv + 1024) * G * (d + 2) * 4 bytes, which fits up to that limit for
- *   G = 8, d = 128 -- and for shapes the decode kernel does not serve. No device-side status is kept:
- *   lengths that do not fit the cache are skipped without a report. */
+ *   G = 8, d = 128 -- and for shapes the decode kernel does not serve. The caller
+ *   cannot read the array's status word: lengths that do not fit the cache are
+ *   skipped, and a device wait that runs out (each is bounded at 2 s) leaves that
+ *   call's output rows unspecified, without a report. */
 qsa_status_t qsa_sparse_attn_decode_noalloc(const qsa_config_t *cfg, const void *q, const void *k,
                                             const void *v, const int32_t *sel, const int32_t *kv_start,
                                             const int32_t *kv_len, int32_t batch, int32_t kv_cap, void *out,

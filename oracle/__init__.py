@@ -237,6 +237,29 @@ def scores(cfg, inp: Dict[str, torch.Tensor], b: int, r_idx: Sequence[int],
     return out[:, :nb]
 
 
+def attend_selection(cfg, inp: Dict[str, torch.Tensor], b: int, r_idx: Sequence[int],
+                     sel_rows: np.ndarray, decode: Optional[bool] = None) -> np.ndarray:
+    """fp64 attention outputs [len(r_idx)][Hq][d] of sequence b's query rows r_idx over
+    the token sets that the given selections (sel_rows [len(r_idx)][k], e.g. another
+    implementation's) define, together with each row's trailing range."""
+    if decode is None:
+        decode = "k_new" in inp
+    scale = getattr(cfg, "scale", None) or 1.0 / float(np.sqrt(cfg.d))
+    k, v, _, L = _sequence_views(inp, b, decode)
+    ka, dt = _raw(k)
+    va, _ = _raw(v)
+    out = np.zeros((len(r_idx), cfg.Hq, cfg.d), dtype=np.float64)
+    for i, r in enumerate(r_idx):
+        t = int(r) + int(inp["q_first"][b])
+        toks = token_set(t, cfg.block, np.asarray(sel_rows[i], dtype=np.int32))
+        qa, _ = _raw(inp["q"][b, r])
+        o = np.zeros((cfg.Hq, cfg.d), dtype=np.float64)
+        lib().qsa_oracle_attend(_ptr(qa), _ptr(ka), _ptr(va), dt, cfg.Hq, cfg.Hkv, cfg.d, L, scale,
+                                toks.ctypes.data_as(_I64), toks.shape[0], _dptr(o))
+        out[i] = o
+    return out
+
+
 class use_library:
     """Context manager: route oracle calls to another build of qsa_oracle.c (used by
     the mutation test, which plants mistakes in a copy of the oracle on the CPU)."""

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(qsa):
 
 
 def test_abi_version_and_status_strings(qsa):
-    assert qsa.qsa_abi_version() == 1
+    assert qsa.qsa_abi_version() == 2
     for s in range(6):
         assert qsa.status_string(s)
     assert qsa.status_string(99) == "unknown status"
@@ -90,7 +90,7 @@ def test_null_and_misaligned_pointers_rejected_on_host(qsa):
                              None) == qsa.QSA_ERR_INVALID_ARG
     assert L.qsa_index_score_topk(cp, None, None, None, None, 1, 16, 16, None, None, 1 << 20,
                                   None) == qsa.QSA_ERR_INVALID_ARG
-    assert L.qsa_compress_blocks(cp, None, None, None, None, 1, 64, None, None) == qsa.QSA_ERR_INVALID_ARG
+    assert L.qsa_compress_blocks(cp, None, None, None, None, 1, 64, None, None, None) == qsa.QSA_ERR_INVALID_ARG
     assert L.qsa_forward(cp, qsa.QSA_PREFILL, None, None, 0, None) == qsa.QSA_ERR_INVALID_ARG
     # misaligned (never dereferenced: rejected before any launch)
     bad = P(0x1001)

@@ -13,11 +13,13 @@ WL = W.WORKLOADS
 
 
 def run_prefill(qsa, w, inp):
+    """qsa_forward(PREFILL) with guard bands around out and sel, checked after the call."""
     from block_sparse_long_15_b200.runner import QSAPrefill
-    p = QSAPrefill(w, inp)
+    p = QSAPrefill(w, inp, guard=True)
     out, sel = p()
     torch.cuda.synchronize()
     assert p.status() == qsa.QSA_OK
+    assert p.guards_intact(), "a kernel wrote outside out / sel"
     return out.cpu(), sel.cpu(), p
 
 
@@ -26,21 +28,33 @@ def oracle_rows(w, inp, n_random, seed):
                            n_random, seed + b) for b in range(w.batch)}
 
 
+def assert_kbar_close(g, o):
+    """Compressed keys: the kernel's fp32 block means against the oracle's fp64 ones,
+    |g - o| <= 1e-6 + 1e-5 |o| (an fp32 sum of B bf16/fp32 keys in key order, then a
+    division by B, is within a few fp32 ulps of the exact mean)."""
+    g = g.double().cpu().numpy()
+    assert g.shape == o.shape, (g.shape, o.shape)
+    err = np.abs(g - o) - (1e-6 + 1e-5 * np.abs(o))
+    assert err.max() <= 0, f"kbar off by {np.abs(g - o).max():.3e}"
+
+
 def assert_report(rep, w, max_near_tie_frac=0.01):
     print(w.name, rep)
     assert rep.ok(), str(rep)
     assert rep.near_tie_rows <= max(1, max_near_tie_frac * rep.rows), str(rep)
+    assert rep.near_tie_checked == rep.near_tie_rows, str(rep)
 
 
 # ----------------------------------------------------------------------------- fp32 tiny
 def test_tiny_fp32_full(cuda_lib):
     w = WL["tiny_fp32_prefill_s256"]
     inp = W.make_inputs(w)
-    out, sel, _ = run_prefill(cuda_lib, w, inp)
-    orc = oracle.run(w, inp)
+    out, sel, p = run_prefill(cuda_lib, w, inp)
+    orc = oracle.run(w, inp, want_kbar=True)
     rep = compare(w, inp, out, sel, orc)
     assert_report(rep, w, 0.0)
     assert rep.sel_exact == rep.rows == 256
+    assert_kbar_close(p.t["kbar_cache"][0, : 256 // w.block], orc["kbar"][0])
 
 
 # ----------------------------------------------------------------------------- bf16 prefill
@@ -49,9 +63,11 @@ def test_bf16_prefill_small_full_rows(cuda_lib, seq):
     """Every row at sizes spanning several tiles and a ragged tail."""
     w = W.small_variant(WL["bf16_prefill_s8192"], seq=seq)
     inp = W.make_inputs(w)
-    out, sel, _ = run_prefill(cuda_lib, w, inp)
-    rep = compare(w, inp, out, sel, oracle.run(w, inp))
+    out, sel, p = run_prefill(cuda_lib, w, inp)
+    orc = oracle.run(w, inp, want_kbar=True)
+    rep = compare(w, inp, out, sel, orc)
     assert_report(rep, w)
+    assert_kbar_close(p.t["kbar_cache"][0, : seq // w.block], orc["kbar"][0])
 
 
 def test_bf16_prefill_s8192_sampled(cuda_lib):
@@ -86,9 +102,13 @@ def test_varlen_leftpad_full_size_sampled(cuda_lib):
 def test_varlen_leftpad_small_full_rows(cuda_lib):
     w = W.small_variant(WL["bf16_prefill_varlen_b8_s16384_leftpad"], seq=700, batch=3, pad_max=300)
     inp = W.make_inputs(w)
-    out, sel, _ = run_prefill(cuda_lib, w, inp)
-    rep = compare(w, inp, out, sel, oracle.run(w, inp))
+    out, sel, p = run_prefill(cuda_lib, w, inp)
+    orc = oracle.run(w, inp, want_kbar=True)
+    rep = compare(w, inp, out, sel, orc)
     assert_report(rep, w)
+    for b in range(w.batch):  # k̄ rows count from each sequence's first real token
+        n_blk = int(inp["kv_len"][b]) // w.block
+        assert_kbar_close(p.t["kbar_cache"][b, :n_blk], orc["kbar"][b])
 
 
 # ----------------------------------------------------------------------------- edge cases
@@ -144,10 +164,11 @@ def test_decode_b64_full(cuda_lib):
     from block_sparse_long_15_b200.runner import QSADecode
     w = WL["bf16_decode_b64_l4k_32k"]
     inp = W.make_inputs(w)
-    d = QSADecode(w, inp)
+    d = QSADecode(w, inp, guard=True)
     out, sel = d()
     torch.cuda.synchronize()
     assert d.status() == cuda_lib.QSA_OK
+    assert d.guards_intact()
     orc = oracle.run(w, inp)
     rep = compare(w, inp, out.cpu(), sel.cpu(), orc, decode=True)
     assert_report(rep, w, 0.05)
