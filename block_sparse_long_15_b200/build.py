@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libqsa.so")
 SOURCES = ["qsa_api.cu", "qsa_simt.cu", "qsa_score_tc.cu", "qsa_attn_tc.cu", "qsa_attn_tc1.cu", "qsa_decode.cu",
-           "qsa_offload.cu", "qsa_selftest.cu"]
+           "qsa_offload.cu", "qsa_selftest.cu", "qsa_proj.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
                 "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -304,6 +304,65 @@ qsa_status_t qsa_index_score_topk(const qsa_config_t *cfg, const void *qi, const
   return score_dispatch(D, S, qi, kbar, sel, workspace, (cudaStream_t)stream);
 }
 
+qsa_status_t qsa_project(const qsa_config_t *cfg, const qsa_proj_config_t *pc, const void *x, const void *w,
+                         const int32_t *q_first, int32_t batch, int32_t n_tok, void *q, void *qi, void *k,
+                         void *v, void *ki, int32_t kv_cap, int32_t kv_row0, void *workspace,
+                         size_t workspace_bytes, qsa_stream_t stream) {
+  g_serial_at_entry = g_error_serial;
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if (!pc || batch < 0 || n_tok < 0 || kv_cap < 0 || kv_row0 < 0) return QSA_ERR_INVALID_ARG;
+  if (batch == 0 || n_tok == 0) return QSA_OK;
+  if ((long long)kv_row0 + n_tok > kv_cap) return QSA_ERR_INVALID_ARG;
+  if (!(pc->rope_theta > 0.f) || pc->hidden_size <= 0) return QSA_ERR_INVALID_ARG;
+  if (!proj_supported(D, pc->hidden_size, pc->rotary_dim, pc->indexer_rotary_dim)) return QSA_ERR_UNSUPPORTED;
+  if (!x || !w || !q_first || !q || !qi || !k || !v || !ki || !workspace) return QSA_ERR_INVALID_ARG;
+  const void *ptrs[] = {x, w, q, qi, k, v, ki, workspace};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return QSA_ERR_INVALID_ARG;
+  if (workspace_bytes < kStatusBytes) return QSA_ERR_INVALID_ARG;
+  return cuda_status(launch_proj_rope(D, pc->hidden_size, pc->rope_theta, pc->rotary_dim, pc->indexer_rotary_dim,
+                                      x, w, q_first, batch, n_tok, q, qi, k, v, ki, kv_cap, kv_row0,
+                                      status_word(workspace), (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_index_scores(const qsa_config_t *cfg, const void *qi, const float *kbar, const int32_t *kv_len,
+                              const int32_t *q_first, int32_t batch, int32_t n_q, int32_t kv_cap, float *scores,
+                              void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+  g_serial_at_entry = g_error_serial;
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if ((s = check_sizes(D, batch, n_q, kv_cap)) != QSA_OK) return s;
+  if (batch == 0 || n_q == 0 || kv_cap / D.B == 0) return QSA_OK;  // no complete block: nothing to score
+  if (!qi || !kbar || !kv_len || !q_first || !scores || !workspace) return QSA_ERR_INVALID_ARG;
+  if (!aligned16(qi) || !aligned16(kbar) || !aligned16(scores) || !aligned16(workspace)) return QSA_ERR_INVALID_ARG;
+  Seqs S = make_seqs(D, nullptr, kv_len, q_first, batch, n_q, kv_cap);
+  if (workspace_bytes < kStatusBytes + scratch_need(D, S)) return QSA_ERR_INVALID_ARG;
+  int *status = status_word(workspace);
+  if (use_score_tc(D, S))
+    return cuda_status(launch_score_topk_tc(D, S, qi, kbar, nullptr, (char *)workspace + kStatusBytes, status,
+                                            (cudaStream_t)stream, scores));
+  return cuda_status(launch_index_scores_simt(D, S, qi, kbar, scores, status, (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_select_topk(const qsa_config_t *cfg, const float *scores, const int32_t *kv_len,
+                             const int32_t *q_first, int32_t batch, int32_t n_q, int32_t kv_cap, int32_t *sel,
+                             void *workspace, size_t workspace_bytes, qsa_stream_t stream) {
+  g_serial_at_entry = g_error_serial;
+  Dims D;
+  qsa_status_t s = resolve(cfg, &D);
+  if (s != QSA_OK) return s;
+  if ((s = check_sizes(D, batch, n_q, kv_cap)) != QSA_OK) return s;
+  if (batch == 0 || n_q == 0) return QSA_OK;
+  if ((!scores && kv_cap / D.B > 0) || !kv_len || !q_first || !sel || !workspace) return QSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(sel) || !aligned16(workspace)) return QSA_ERR_INVALID_ARG;
+  if (workspace_bytes < kStatusBytes) return QSA_ERR_INVALID_ARG;
+  Seqs S = make_seqs(D, nullptr, kv_len, q_first, batch, n_q, kv_cap);
+  return cuda_status(launch_select_topk(D, S, scores, sel, status_word(workspace), (cudaStream_t)stream));
+}
+
 qsa_status_t qsa_sparse_attn(const qsa_config_t *cfg, const void *q, const void *k, const void *v,
                              const int32_t *sel, const int32_t *kv_start, const int32_t *kv_len,
                              const int32_t *q_first, int32_t batch, int32_t n_q, int32_t kv_cap,

@@ -118,6 +118,12 @@ struct DecodeAppend {
 cudaError_t launch_decode_append_score(const Dims &D, const Seqs &S, const DecodeAppend &A, const void *qi,
                                        float *kbar, int32_t *sel, int *status, cudaStream_t st);
 
+// Input projections with RoPE (tcgen05 GEMM, bf16): see qsa_project in qsa.h.
+bool proj_supported(const Dims &D, int hidden, int rd_attn, int rd_idx);
+cudaError_t launch_proj_rope(const Dims &D, int hidden, float rope_theta, int rd_attn, int rd_idx, const void *x,
+                             const void *w, const int32_t *pos0, int batch, int n_tok, void *q, void *qi, void *k,
+                             void *v, void *ki, int kv_cap, int kv_row0, int *status, cudaStream_t st);
+
 // Step 4 on CUDA cores (fp32 accumulate), any supported shape.
 cudaError_t launch_attn_simt(const Dims &D, const Seqs &S, const void *q, const void *k,
                              const void *v, const int32_t *sel, void *out, int *status,

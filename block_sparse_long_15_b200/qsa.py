@@ -37,6 +37,11 @@ class qsa_config_t(ctypes.Structure):
                 ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
 
 
+class qsa_proj_config_t(ctypes.Structure):
+    _fields_ = [("hidden_size", ctypes.c_int32), ("rope_theta", ctypes.c_float), ("rotary_dim", ctypes.c_int32),
+                ("indexer_rotary_dim", ctypes.c_int32)]
+
+
 class qsa_tensors_t(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_q", ctypes.c_int32), ("kv_cap", ctypes.c_int32),
                 ("q", ctypes.c_void_p), ("qi", ctypes.c_void_p), ("k_cache", ctypes.c_void_p),
@@ -62,6 +67,9 @@ def _load() -> ctypes.CDLL:
         "qsa_compress_blocks": ([cfgp, V, V, V, V, I, I, V, V, V], I),
         "qsa_index_score_topk": ([cfgp, V, V, V, V, I, I, I, V, V, S, V], I),
         "qsa_sparse_attn": ([cfgp, V, V, V, V, V, V, V, I, I, I, V, V, S, V], I),
+        "qsa_index_scores": ([cfgp, V, V, V, V, I, I, I, V, V, S, V], I),
+        "qsa_project": ([cfgp, P(qsa_proj_config_t), V, V, V, I, I, V, V, V, V, V, I, I, V, S, V], I),
+        "qsa_select_topk": ([cfgp, V, V, V, I, I, I, V, V, S, V], I),
         "qsa_forward": ([cfgp, I, P(qsa_tensors_t), V, S, V], I),
         "qsa_read_device_status": ([V, V, P(I)], I),
         "qsa_abi_version": ([], I),
@@ -85,7 +93,8 @@ EXPORTED = ("qsa_config_validate", "qsa_topk_blocks", "qsa_status_string", "qsa_
             "qsa_compress_blocks", "qsa_index_score_topk", "qsa_sparse_attn", "qsa_forward",
             "qsa_read_device_status", "qsa_abi_version", "qsa_attn_kernel_name",
             "qsa_kernel_launch_count", "qsa_last_error", "qsa_sparse_attn_decode_noalloc",
-            "qsa_selftest_wait_timeout", "qsa_offload_staging_size", "qsa_decode_offload")
+            "qsa_selftest_wait_timeout", "qsa_offload_staging_size", "qsa_decode_offload",
+            "qsa_index_scores", "qsa_select_topk", "qsa_project")
 
 # Size of the library's fixed decode scratch (QSA_NOALLOC_SCRATCH_BYTES in qsa.h).
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -215,6 +224,55 @@ def qsa_index_score_topk(cfg, qi, kbar, kv_len, q_first, kv_cap, sel, workspace,
     _check(_lib.qsa_index_score_topk(ctypes.byref(cfg), _p(qi), _p(kbar), _p(kv_len), _p(q_first), batch,
                                      n_q, kv_cap, _p(sel), _p(workspace), workspace.numel(),
                                      _stream(stream)), "qsa_index_score_topk")
+
+
+def qsa_project(cfg, pc: qsa_proj_config_t, x, w, q_first, q, qi, k, v, ki, kv_row0: int = 0, workspace=None,
+                stream=None):
+    """Projections of x [batch][n_tok][D] by the stacked weights w and RoPE, written to
+    q [batch][n_tok][Hq][d], qi [batch][n_tok][Hi][di], k / v [batch][Hkv][kv_cap][d] and
+    ki [batch][kv_cap][di] (rows kv_row0 + r)."""
+    batch, n_tok, D = x.shape
+    kv_cap = k.shape[2]
+    n_out = (cfg.num_attention_heads * cfg.head_dim + 2 * cfg.num_key_value_heads * cfg.head_dim
+             + cfg.indexer_n_heads * cfg.indexer_head_dim + cfg.indexer_head_dim)
+    dt = _elem(cfg)
+    _want(x, dt, (batch, n_tok, pc.hidden_size), "x")
+    _want(w, dt, (n_out, pc.hidden_size), "w")
+    _want(q, dt, (batch, n_tok, cfg.num_attention_heads, cfg.head_dim), "q")
+    _want(qi, dt, (batch, n_tok, cfg.indexer_n_heads, cfg.indexer_head_dim), "qi")
+    _want(k, dt, (batch, cfg.num_key_value_heads, kv_cap, cfg.head_dim), "k")
+    _want(v, dt, (batch, cfg.num_key_value_heads, kv_cap, cfg.head_dim), "v")
+    _want(ki, dt, (batch, kv_cap, cfg.indexer_head_dim), "ki")
+    _want_lengths(batch, q_first=q_first)
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=x.device)
+    _check(_lib.qsa_project(ctypes.byref(cfg), ctypes.byref(pc), _p(x), _p(w), _p(q_first), batch, n_tok, _p(q),
+                            _p(qi), _p(k), _p(v), _p(ki), kv_cap, kv_row0, _p(workspace), workspace.numel(),
+                            _stream(stream)), "qsa_project")
+    return workspace
+
+
+def qsa_index_scores(cfg, qi, kbar, kv_len, q_first, kv_cap, scores, workspace, stream=None):
+    """Scores over the heads in qi (a shard of the indexer query heads), written to
+    scores [batch][n_q][kv_cap // B] fp32 for each real row's candidate blocks."""
+    batch, n_q = qi.shape[0], qi.shape[1]
+    nb = kv_cap // cfg.indexer_compress_ratio
+    _want(qi, _elem(cfg), (batch, n_q, cfg.indexer_n_heads, cfg.indexer_head_dim), "qi")
+    _want(kbar, torch.float32, (batch, nb, cfg.indexer_head_dim), "kbar")
+    _want(scores, torch.float32, (batch, n_q, nb), "scores")
+    _want_lengths(batch, kv_len=kv_len, q_first=q_first)
+    _check(_lib.qsa_index_scores(ctypes.byref(cfg), _p(qi), _p(kbar), _p(kv_len), _p(q_first), batch, n_q, kv_cap,
+                                 _p(scores), _p(workspace), workspace.numel(), _stream(stream)), "qsa_index_scores")
+
+
+def qsa_select_topk(cfg, scores, kv_len, q_first, kv_cap, sel, workspace, stream=None):
+    """Top-k blocks of each real row from a score matrix [batch][n_q][kv_cap // B] fp32."""
+    batch, n_q = scores.shape[0], scores.shape[1]
+    _want(scores, torch.float32, (batch, n_q, kv_cap // cfg.indexer_compress_ratio), "scores")
+    _want(sel, torch.int32, (batch, n_q, qsa_topk_blocks(cfg)), "sel")
+    _want_lengths(batch, kv_len=kv_len, q_first=q_first)
+    _check(_lib.qsa_select_topk(ctypes.byref(cfg), _p(scores), _p(kv_len), _p(q_first), batch, n_q, kv_cap, _p(sel),
+                                _p(workspace), workspace.numel(), _stream(stream)), "qsa_select_topk")
 
 
 def qsa_sparse_attn(cfg, q, k, v, sel, kv_start, kv_len, q_first, out, workspace, stream=None):

@@ -167,6 +167,62 @@ qsa_status_t qsa_sparse_attn(const qsa_config_t *cfg, const void *q, const void 
                              void *out, void *workspace, size_t workspace_bytes,
                              qsa_stream_t stream);
 
+/* The steps before the path: input projections and rotary position embedding
+ * ("Qwen4-Exp" Qwen4ExpTextConfig: hidden_size; attention_bias = False, so no bias;
+ * rope_parameters holding rope_theta; the head counts and dims of qsa_config_t).
+ * Readings (the page fixes neither): RoPE in rotate-half form on the first rotary_dim
+ * dims of every q and k head -- dims (i, i + r/2), i < r/2, turn by
+ * pos * rope_theta^(-2i/r) -- and, with indexer_rotary_dim > 0, likewise on the
+ * indexer query heads and the indexer key head; v is never rotated. */
+typedef struct {
+  int32_t hidden_size;        /* D: length of an input row and of every weight row; multiple of 64 */
+  float rope_theta;           /* base of the rotary frequencies (rope_parameters["rope_theta"]) */
+  int32_t rotary_dim;         /* dims of each q / k head that rotate: multiple of 32, <= head_dim */
+  int32_t indexer_rotary_dim; /* same for the indexer heads (<= indexer_head_dim); 0: they do not rotate */
+} qsa_proj_config_t;
+
+/* Projects the token rows x [batch][n_tok][D] (bf16) by the stacked weight rows
+ * w [Hq*d + 2*Hkv*d + Hi*di + di][D] (bf16: W_q, W_k, W_v, W_qi, W_ki one after the
+ * other, each [out][D]) in fp32, applies RoPE at position q_first[b] + r to token row r
+ * of sequence b, and writes bf16: q [batch][n_tok][Hq][d], qi [batch][n_tok][Hi][di],
+ * and k, v [batch][Hkv][kv_cap][d], ki [batch][kv_cap][di] at storage row kv_row0 + r.
+ * Prefill: q_first as for qsa_forward (-pad), kv_cap = n_tok, kv_row0 = 0. A decode
+ * step: n_tok = 1, q_first[b] = kv_len[b] - 1, and k / v / ki are qsa_tensors_t's
+ * k_new / v_new / ki_new (kv_cap = 1, kv_row0 = 0). Runs on tcgen05 tensor cores;
+ * bf16 only, head_dim and indexer_head_dim multiples of 64 up to 256. Returns
+ * QSA_ERR_UNSUPPORTED for other shapes. workspace: at least the 256-byte status word. */
+qsa_status_t qsa_project(const qsa_config_t *cfg, const qsa_proj_config_t *pc, const void *x, const void *w,
+                         const int32_t *q_first, int32_t batch, int32_t n_tok, void *q, void *qi, void *k,
+                         void *v, void *ki, int32_t kv_cap, int32_t kv_row0, void *workspace,
+                         size_t workspace_bytes, qsa_stream_t stream);
+
+/* Head-sharded tensor parallelism ("Qwen4-Exp" Usage tips: tp_plan="auto" shards QSA;
+ * the QSA projection dims must be divisible by the TP size). The block score is a sum
+ * over indexer heads, so a rank holding a shard of the indexer query heads computes a
+ * partial score; the partials summed over ranks (an all-reduce of the score matrix,
+ * the caller's collective) are the full scores, from which every rank selects the same
+ * blocks and attends its own shard of query / KV heads with qsa_sparse_attn.
+ *
+ * qsa_index_scores: step 2 alone. With cfg describing this rank's shard
+ * (indexer_n_heads = the shard's head count, qi holding those heads), writes
+ * scores[b][r][j] = sum over the shard's heads h of max(0, qi[b][r][h] . kbar[b][j])
+ * for j < n_c(t) of every real query row; entries j >= n_c(t) and padding rows are not
+ * written (they are never read by qsa_select_topk). Layout scores [batch][n_q][kv_cap / B]
+ * fp32, device memory, 16-byte aligned. bf16 shapes with many rows run on the tensor
+ * cores with the same precision as qsa_index_score_topk (kbar as a bf16 hi/lo pair);
+ * others in fp32 on CUDA cores. workspace as for qsa_index_score_topk.
+ *
+ * qsa_select_topk: step 3 alone. Reads each real row's n_c(t) scores (any finite
+ * fp32 values; -0 counts as +0) and writes sel[b][r][0..k) exactly as
+ * qsa_index_score_topk does: the k best blocks by (-score, block id), ascending, -1
+ * padded; padding rows all -1. workspace: at least the 256-byte status word. */
+qsa_status_t qsa_index_scores(const qsa_config_t *cfg, const void *qi, const float *kbar, const int32_t *kv_len,
+                              const int32_t *q_first, int32_t batch, int32_t n_q, int32_t kv_cap, float *scores,
+                              void *workspace, size_t workspace_bytes, qsa_stream_t stream);
+qsa_status_t qsa_select_topk(const qsa_config_t *cfg, const float *scores, const int32_t *kv_len,
+                             const int32_t *q_first, int32_t batch, int32_t n_q, int32_t kv_cap, int32_t *sel,
+                             void *workspace, size_t workspace_bytes, qsa_stream_t stream);
+
 /* The whole path.
  * QSA_PREFILL: compress every complete block of each prompt into kbar_cache (and set
  *   kbar_blocks[b] = kv_len[b] / B), then score, select and attend all n_q query rows.

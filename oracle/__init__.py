@@ -71,6 +71,11 @@ def lib():
                                                      ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                      ctypes.c_int, _D, ctypes.c_int]
             L.qsa_oracle_max_threads.restype = ctypes.c_int
+            L.qsa_oracle_rope_head.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double]
+            L.qsa_oracle_project_rope.argtypes = [_V, _V, ctypes.c_int, ctypes.c_int64, ctypes.c_int, _I64,
+                                                  ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _D,
+                                                  ctypes.c_int]
             _lib = L
     return _lib
 
@@ -237,6 +242,39 @@ def scores(cfg, inp: Dict[str, torch.Tensor], b: int, r_idx: Sequence[int],
     return out[:, :nb]
 
 
+def rope_head(h, pos: float, theta: float, rd: int) -> np.ndarray:
+    """One head vector rotated at position pos (rotate-half form, first rd dims)."""
+    out = np.ascontiguousarray(np.asarray(h, dtype=np.float64).copy())
+    lib().qsa_oracle_rope_head(_dptr(out), out.shape[0], rd, float(pos), float(theta))
+    return out
+
+
+def project_rope(pc, x, w, pos, n_threads: int = 0) -> Dict[str, np.ndarray]:
+    """Projections of the rows x [n][D] by the stacked weights w [n_out][D] and RoPE at
+    positions pos [n]. pc: Hq, Hkv, d, Hi, di, rope_theta, rd_attn, rd_idx.
+    Returns fp64 q [n][Hq][d], k [n][Hkv][d], v [n][Hkv][d], qi [n][Hi][di], ki [n][di]."""
+    xa, dt = _raw(x)
+    wa, dt2 = _raw(w)
+    assert dt == dt2
+    n, D = xa.shape
+    n_out = pc.Hq * pc.d + 2 * pc.Hkv * pc.d + pc.Hi * pc.di + pc.di
+    assert wa.shape == (n_out, D), (wa.shape, n_out, D)
+    p = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    y = np.zeros((n, n_out), dtype=np.float64)
+    lib().qsa_oracle_project_rope(_ptr(xa), _ptr(wa), dt, n, D, p.ctypes.data_as(_I64), float(pc.rope_theta),
+                                  pc.Hq, pc.Hkv, pc.d, pc.Hi, pc.di, pc.rd_attn, pc.rd_idx, _dptr(y), n_threads)
+    a, b = 0, pc.Hq * pc.d
+    out = {"q": y[:, a:b].reshape(n, pc.Hq, pc.d)}
+    a, b = b, b + pc.Hkv * pc.d
+    out["k"] = y[:, a:b].reshape(n, pc.Hkv, pc.d)
+    a, b = b, b + pc.Hkv * pc.d
+    out["v"] = y[:, a:b].reshape(n, pc.Hkv, pc.d)
+    a, b = b, b + pc.Hi * pc.di
+    out["qi"] = y[:, a:b].reshape(n, pc.Hi, pc.di)
+    out["ki"] = y[:, b:b + pc.di]
+    return out
+
+
 def attend_selection(cfg, inp: Dict[str, torch.Tensor], b: int, r_idx: Sequence[int],
                      sel_rows: np.ndarray, decode: Optional[bool] = None) -> np.ndarray:
     """fp64 attention outputs [len(r_idx)][Hq][d] of sequence b's query rows r_idx over
@@ -275,7 +313,8 @@ class use_library:
         other = ctypes.CDLL(self.path)
         for name in ("qsa_oracle_compress", "qsa_oracle_block_scores", "qsa_oracle_select",
                      "qsa_oracle_token_set", "qsa_oracle_attend", "qsa_oracle_sequence",
-                     "qsa_oracle_sequence_scores", "qsa_oracle_max_threads"):
+                     "qsa_oracle_sequence_scores", "qsa_oracle_max_threads", "qsa_oracle_rope_head",
+                     "qsa_oracle_project_rope"):
             f, g = getattr(saved, name), getattr(other, name)
             g.argtypes, g.restype = f.argtypes, f.restype
         self.saved = saved

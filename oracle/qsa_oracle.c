@@ -271,6 +271,64 @@ void qsa_oracle_sequence_scores(const void *qi, const int64_t *t_pos, int64_t n_
     free(kbar);
 }
 
+/*
+ * Input projections and rotary position embedding, the steps before the path
+ * (Qwen4ExpTextConfig: hidden_size, attention_bias = False so no bias terms,
+ * rope_parameters with rope_theta; num_attention_heads / num_key_value_heads /
+ * head_dim for q, k, v; indexer_n_heads / indexer_head_dim for the indexer query
+ * heads and the single indexer key head).
+ *
+ * One rotary head of dimension hd at position pos, in place, rotate-half form
+ * (readings: the page fixes neither the pairing nor the rotary fraction): the
+ * first rd dims rotate (rd even, <= hd); for i < rd / 2, with
+ * angle_i = pos * theta^(-2 i / rd), the pair (h[i], h[i + rd/2]) becomes
+ * (h[i] cos - h[i + rd/2] sin, h[i + rd/2] cos + h[i] sin); dims >= rd are kept.
+ */
+void qsa_oracle_rope_head(double *h, int hd, int rd, double pos, double theta) {
+    (void)hd;
+    int half = rd / 2;
+    for (int i = 0; i < half; ++i) {
+        double ang = pos * pow(theta, -2.0 * (double)i / (double)rd);
+        double c = cos(ang), sn = sin(ang);
+        double a = h[i], b = h[i + half];
+        h[i] = a * c - b * sn;
+        h[i + half] = b * c + a * sn;
+    }
+}
+
+/*
+ * y[r][o] = sum_c x[r][c] w[o][c] for the stacked weight rows
+ *   [W_q: Hq*d][W_k: Hkv*d][W_v: Hkv*d][W_qi: Hi*di][W_ki: di]   (n_out rows of D)
+ * then RoPE at position pos[r] on every q and k head (rotary dims rd_attn) and on
+ * every indexer query head and the indexer key head (rotary dims rd_idx; 0 = none);
+ * v is never rotated.  x [n_rows][D] and w in fp32 or bf16 (dtype), y fp64.
+ */
+void qsa_oracle_project_rope(const void *x, const void *w, int dtype, int64_t n_rows, int D,
+                             const int64_t *pos, double theta, int Hq, int Hkv, int d, int Hi,
+                             int di, int rd_attn, int rd_idx, double *y, int n_threads) {
+    int n_out = Hq * d + 2 * Hkv * d + Hi * di + di;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        double *yr = y + (size_t)r * n_out;
+        for (int o = 0; o < n_out; ++o) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c)
+                acc += orc_load(x, dtype, (size_t)r * D + c) * orc_load(w, dtype, (size_t)o * D + c);
+            yr[o] = acc;
+        }
+        double p = (double)pos[r];
+        for (int h = 0; h < Hq + Hkv; ++h) qsa_oracle_rope_head(yr + (size_t)h * d, d, rd_attn, p, theta);
+        double *yi = yr + (size_t)(Hq + 2 * Hkv) * d;
+        if (rd_idx > 0)
+            for (int h = 0; h < Hi + 1; ++h) qsa_oracle_rope_head(yi + (size_t)h * di, di, rd_idx, p, theta);
+    }
+}
+
 int qsa_oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

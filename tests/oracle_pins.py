@@ -316,4 +316,75 @@ def pin_selection_scale_invariance(orc):
         assert np.array_equal(a["sel"][0], b["sel"][0]), key
 
 
+# --------------------------------------------------------------------------- projections + RoPE
+def _pc(**kw):
+    base = dict(Hq=4, Hkv=2, d=8, Hi=2, di=4, rope_theta=100.0, rd_attn=8, rd_idx=4)
+    base.update(kw)
+    return types.SimpleNamespace(**base)
+
+
+def _proj_inputs(pc, n, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    n_out = pc.Hq * pc.d + 2 * pc.Hkv * pc.d + pc.Hi * pc.di + pc.di
+    return torch.randn(n, D, generator=g), torch.randn(n_out, D, generator=g) * 0.3
+
+
+def pin_projection_is_the_matmul_at_position_zero(orc):
+    """At position 0 every rotation is the identity: the stage is x W^T (library matmul
+    in fp64), split into q, k, v, qi, ki by the stacked-row layout."""
+    pc = _pc()
+    x, w = _proj_inputs(pc, 5, 12, 0)
+    out = orc.project_rope(pc, x, w, [0] * 5)
+    y = (x.double() @ w.double().T).numpy()
+    flat = np.concatenate([out["q"].reshape(5, -1), out["k"].reshape(5, -1), out["v"].reshape(5, -1),
+                           out["qi"].reshape(5, -1), out["ki"]], axis=1)
+    assert np.allclose(flat, y, rtol=1e-12, atol=1e-12)
+
+
+def pin_rope_hand_worked(orc):
+    """Head [1, 0, 0, 0], rd 4, theta 100: dim 0 pairs with dim 2 at frequency 1, dim 1
+    with dim 3 at frequency 100^(-1/2) = 0.1. At pos pi/2 the first pair turns a
+    quarter: [0, 0, 1, 0]; [0, 1, 0, 0] at pos 5 turns by 0.5 rad: [0, cos .5, 0, sin .5]."""
+    a = orc.rope_head([1, 0, 0, 0], math.pi / 2, 100.0, 4)
+    assert np.allclose(a, [0, 0, 1, 0], atol=1e-15), a
+    b = orc.rope_head([0, 1, 0, 0], 5.0, 100.0, 4)
+    assert np.allclose(b, [0, math.cos(0.5), 0, math.sin(0.5)], atol=1e-15), b
+    c = orc.rope_head([0, 0, 2, 0], 1.0, 100.0, 4)  # the second half rotates the other way
+    assert np.allclose(c, [-2 * math.sin(1.0), 0, 2 * math.cos(1.0), 0], atol=1e-15), c
+
+
+def pin_rope_norm_and_relative_position(orc):
+    """A rotation keeps each head's norm, and q . k after RoPE depends only on the
+    distance between the two positions."""
+    g = np.random.default_rng(3)
+    q, k = g.standard_normal(16), g.standard_normal(16)
+    for p in (0, 1, 7, 1000):
+        assert abs(np.linalg.norm(orc.rope_head(q, p, 1e4, 16)) - np.linalg.norm(q)) < 1e-12
+    d1 = orc.rope_head(q, 9, 1e4, 16) @ orc.rope_head(k, 4, 1e4, 16)
+    d2 = orc.rope_head(q, 1009, 1e4, 16) @ orc.rope_head(k, 1004, 1e4, 16)
+    d3 = orc.rope_head(q, 9, 1e4, 16) @ orc.rope_head(k, 5, 1e4, 16)
+    assert abs(d1 - d2) < 1e-10 and abs(d1 - d3) > 1e-3, (d1, d2, d3)
+
+
+def pin_rope_partial_and_which_heads(orc):
+    """With rotary dims rd < d only the first rd dims of a head move; v is never
+    rotated; the indexer heads rotate with rd_idx and stay put with rd_idx = 0."""
+    pc = _pc(rd_attn=4, rd_idx=2)
+    x, w = _proj_inputs(pc, 3, 10, 1)
+    at0 = orc.project_rope(pc, x, w, [0, 0, 0])
+    at5 = orc.project_rope(pc, x, w, [5, 5, 5])
+    for name in ("q", "k"):
+        assert np.allclose(at5[name][..., 4:], at0[name][..., 4:], atol=1e-12)
+        assert not np.allclose(at5[name][..., :4], at0[name][..., :4])
+    assert np.allclose(at5["v"], at0["v"], atol=1e-12)
+    assert np.allclose(at5["qi"][..., 2:], at0["qi"][..., 2:], atol=1e-12)
+    assert not np.allclose(at5["qi"][..., :2], at0["qi"][..., :2])
+    assert not np.allclose(at5["ki"][..., :2], at0["ki"][..., :2])
+    off = orc.project_rope(_pc(rd_attn=4, rd_idx=0), x, w, [5, 5, 5])
+    assert np.allclose(off["qi"], at0["qi"], atol=1e-12) and np.allclose(off["ki"], at0["ki"], atol=1e-12)
+    # each row rotates at its own position: row 1 of a mixed call equals row 1 at its position alone
+    mixed = orc.project_rope(pc, x, w, [0, 5, 0])
+    assert np.allclose(mixed["q"][1], at5["q"][1], atol=1e-12) and np.allclose(mixed["q"][0], at0["q"][0])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -153,3 +153,23 @@ def test_offload_rejects_null_arguments_on_host(qsa):
     t.batch, t.n_q, t.kv_cap = 2, 1, 4096  # pointers all NULL
     assert lib.qsa_decode_offload(ctypes.byref(c), ctypes.byref(t), None, 0, None, 0, None) == \
         qsa.QSA_ERR_INVALID_ARG
+
+
+def test_project_rejects_bad_arguments_on_host(qsa):
+    L = qsa.library()
+    c = _cfg(qsa)
+    cp = ctypes.byref(c)
+    P = ctypes.c_void_p
+    good = P(0x10000)
+    pc = qsa.qsa_proj_config_t(2048, 1e6, 128, 64)
+    args = lambda pcx, kv_cap=16, row0=0, x=good: (cp, ctypes.byref(pcx), x, good, good, 1, 16, good, good, good,
+                                                   good, good, kv_cap, row0, good, 256, None)
+    assert L.qsa_project(*args(pc, x=P(0x10001))) == qsa.QSA_ERR_INVALID_ARG        # misaligned
+    assert L.qsa_project(*args(pc, kv_cap=8)) == qsa.QSA_ERR_INVALID_ARG             # rows past kv_cap
+    bad_theta = qsa.qsa_proj_config_t(2048, 0.0, 128, 64)
+    assert L.qsa_project(*args(bad_theta)) == qsa.QSA_ERR_INVALID_ARG
+    for bad in (qsa.qsa_proj_config_t(2048, 1e6, 48, 64),    # rotary dim not a multiple of 32
+                qsa.qsa_proj_config_t(2000, 1e6, 128, 64),   # hidden size not a multiple of 64
+                qsa.qsa_proj_config_t(2048, 1e6, 256, 64)):  # more rotary dims than head dims
+        if c.head_dim == 128:
+            assert L.qsa_project(*args(bad)) == qsa.QSA_ERR_UNSUPPORTED

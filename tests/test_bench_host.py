@@ -93,3 +93,26 @@ def test_decode_kernel_bytes_counts_attended_tokens():
         toks = len(oracle.token_set(t, w.block, sel))  # attended tokens of the decode row
         want += toks * w.Hkv * w.d * 2 * 2 + 2 * w.Hq * w.d * 2  # K and V, then q and out (bf16)
     assert bench.decode_kernel_bytes(w, inp) == want
+
+
+def test_executed_tensor_work_model():
+    """k_attn_tc's executed work model: with every block selected, tile i (16 rows of
+    8 heads) multiplies chunks 0 .. (16 i + 15) // 128 of the keys; tiles whose rows
+    select only blocks 1 and 3 (keys 64..127 and 192..255, i.e. chunks 0 and 1) and
+    sit in chunk 3 multiply chunks 0, 1 and 3."""
+    import torch
+    w = W.small_variant(W.WORKLOADS["bf16_prefill_s8192"], seq=512, topk=8)
+    inp = W.make_inputs(w)
+    sel = torch.from_numpy(oracle.run(w, inp)["sel"][0])[None]
+    per = 4 * 128 * 128 * 128 * w.Hkv
+    want = sum((16 * i + 15) // 128 + 1 for i in range(32)) * per
+    assert bench.tc_executed_flops(w, inp, sel) == want
+    w2 = W.small_variant(W.WORKLOADS["bf16_prefill_s8192"], seq=512, topk=2)
+    inp2 = W.make_inputs(w2)
+    sel2 = torch.full((1, 512, 2), -1, dtype=torch.int32)
+    sel2[0, 448:] = torch.tensor([1, 3], dtype=torch.int32)
+    ex = bench.tc_executed_flops(w2, inp2, sel2)
+    # rows 0..447 (tiles 0..27): only their trailing ranges (every id is -1), one chunk each;
+    # tiles 28..31: chunks 0, 1 and the trailing chunk 3
+    want2 = 28 + 4 * 3
+    assert ex == want2 * per, (ex / per, want2)

@@ -29,6 +29,13 @@ MUTANTS = {
     "no_max_subtraction_and_no_norm": ("o_row[(size_t)h * d + c] = n_toks > 0 ? acc / denom : 0.0;",
                                        "o_row[(size_t)h * d + c] = acc;"),
     "selection_keeps_k_minus_1": ("int n_sel = (int)(n_c < k ? n_c : k);", "int n_sel = (int)(n_c < k ? n_c : k - 1);"),
+    "rope_adjacent_pairs": ("double a = h[i], b = h[i + half];\n        h[i] = a * c - b * sn;\n        h[i + half] = b * c + a * sn;",
+                            "double a = h[2 * i], b = h[2 * i + 1];\n        h[2 * i] = a * c - b * sn;\n        h[2 * i + 1] = b * c + a * sn;"),
+    "rope_sin_sign_flipped": ("h[i] = a * c - b * sn;", "h[i] = a * c + b * sn;"),
+    "rope_frequency_exponent_halved": ("pow(theta, -2.0 * (double)i / (double)rd)", "pow(theta, -1.0 * (double)i / (double)rd)"),
+    "rope_rotates_v_too": ("for (int h = 0; h < Hq + Hkv; ++h)", "for (int h = 0; h < Hq + 2 * Hkv; ++h)"),
+    "rope_skips_indexer_key": ("for (int h = 0; h < Hi + 1; ++h)", "for (int h = 0; h < Hi; ++h)"),
+    "projection_transposed_weight": ("orc_load(w, dtype, (size_t)o * D + c)", "orc_load(w, dtype, (size_t)c * n_out + o)"),
 }
 
 
