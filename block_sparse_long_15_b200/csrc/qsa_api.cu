@@ -156,10 +156,10 @@ qsa_status_t cuda_status(cudaError_t e) {
 int *status_word(void *ws) { return (int *)ws; }
 
 qsa_status_t score_dispatch(const Dims &D, const Seqs &S, const void *qi, const float *kbar, int32_t *sel,
-                            void *ws, cudaStream_t st) {
+                            void *ws, cudaStream_t st, bool pdl = false) {
   int *status = (int *)ws;
   if (use_score_tc(D, S))
-    return cuda_status(launch_score_topk_tc(D, S, qi, kbar, sel, (char *)ws + kStatusBytes, status, st));
+    return cuda_status(launch_score_topk_tc(D, S, qi, kbar, sel, (char *)ws + kStatusBytes, status, st, nullptr, pdl));
   return cuda_status(launch_score_topk_simt(D, S, qi, kbar, sel, status, st));
 }
 
@@ -168,12 +168,16 @@ qsa_status_t attn_dispatch(const Dims &D, const Seqs &S, const void *q, const vo
                            bool pdl = false) {
   char *scratch = (char *)ws + kStatusBytes;
   const size_t scratch_bytes = ws_bytes - kStatusBytes;
+#ifdef QSA_DEBUG
+  // debug build: check the selection the attention is about to read
+  if (cudaError_t e = launch_validate_sel(D, S, sel, status_word(ws), st)) return cuda_status(e);
+#endif
   switch (pick_attn(D, S)) {
     case kAttnDecode:
       return cuda_status(
           launch_attn_decode(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st, pdl));
     case kAttnTc:
-      return cuda_status(launch_attn_tc(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st));
+      return cuda_status(launch_attn_tc(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st, pdl));
     case kAttnTc1:
       return cuda_status(launch_attn_tc1(D, S, q, k, v, sel, out, status_word(ws), st));
     default:
@@ -410,10 +414,13 @@ qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensor
   if (workspace_bytes < kStatusBytes + scratch_need(D, S)) return QSA_ERR_INVALID_ARG;
   int *status = status_word(workspace);
   if (mode == QSA_PREFILL) {
+    // compress -> (k̄ split) -> score -> attention, each a programmatic dependent of the
+    // one before: a kernel's prologue overlaps its predecessor's tail, and it waits for
+    // that predecessor before it reads its results
     s = cuda_status(launch_compress(D, S, t->ki_cache, nullptr, t->kbar_cache, t->kbar_blocks,
                                     status, st));
     if (s != QSA_OK) return s;
-    s = score_dispatch(D, S, t->qi, t->kbar_cache, t->sel, workspace, st);
+    s = score_dispatch(D, S, t->qi, t->kbar_cache, t->sel, workspace, st, true);
   } else {
     // The decode query sits at kv_len - 1; a null q_first tells the kernels so.
     S.q_first = nullptr;
@@ -421,10 +428,9 @@ qsa_status_t qsa_forward(const qsa_config_t *cfg, int32_t mode, const qsa_tensor
     s = cuda_status(launch_decode_append_score(D, S, A, t->qi, t->kbar_cache, t->sel, status, st));
   }
   if (s != QSA_OK) return s;
-  // In decode the kernel before the attention is this step's append/selection, which
-  // writes none of the lengths the attention's prologue reads: it may overlap it.
-  return attn_dispatch(D, S, t->q, t->k_cache, t->v_cache, t->sel, t->out, workspace, workspace_bytes, st,
-                       mode == QSA_DECODE);
+  // The kernel before the attention is this call's scoring (prefill) or append and
+  // selection (decode), which writes none of what the attention's prologue reads.
+  return attn_dispatch(D, S, t->q, t->k_cache, t->v_cache, t->sel, t->out, workspace, workspace_bytes, st, true);
 }
 
 

@@ -217,6 +217,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       tma_load_3d(&tm_q, &bars[kBarQ], dst + kQBytes / 2, 64, g * G, z);
     }
   }
+  // sel comes from the kernel before (qsa_forward's scoring, when launched as its
+  // programmatic dependent); everything above read only inputs
+  pdl_wait();
   // Per-tile chunk sets (selected blocks and trailing ranges of the tile's tokens)
   // and a shared-memory copy of the unit's selection lists.
   if (warp >= 2 && has_work) {
@@ -584,7 +587,7 @@ bool attn_tc_supported(const Dims &D) {
 size_t attn_tc_workspace(const Dims &, const Seqs &) { return 0; }
 
 cudaError_t launch_attn_tc(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
-                           const int32_t *sel, void *out, void *, size_t, int *status, cudaStream_t st) {
+                           const int32_t *sel, void *out, void *, size_t, int *status, cudaStream_t st, bool pdl) {
   if (!attn_tc_supported(D)) return cudaErrorNotSupported;
   if (S.batch == 0 || S.n_q == 0) return cudaSuccess;
   CUtensorMap tq, tk, tv;
@@ -617,8 +620,7 @@ cudaError_t launch_attn_tc(const Dims &D, const Seqs &S, const void *q, const vo
   const long long units = (long long)P.n_units * D.Hkv * S.batch;
   if (units > 0x7fffffffLL) return cudaErrorNotSupported;
   note_launch();
-  k_attn_tc<<<(unsigned)units, kThreads, smem, st>>>(tq, tk, tv, P);
-  e = cudaGetLastError();
+  e = launch_maybe_pdl(k_attn_tc, dim3((unsigned)units), dim3(kThreads), smem, st, pdl, tq, tk, tv, P);
   if (e != cudaSuccess) {
     cudaFuncAttributes a;
     char what[160];

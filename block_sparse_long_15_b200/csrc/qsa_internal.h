@@ -77,6 +77,25 @@ cudaError_t ensure_smem(K kernel, size_t bytes) {
   return ensure_smem_for(reinterpret_cast<const void *>(kernel), bytes);
 }
 
+// Launch `kernel` on `st`; with pdl, as a programmatic dependent of the kernel before
+// it in the stream (it may start while that kernel finishes and must griddepcontrol.wait
+// before reading that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                             Args &&...args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&lc, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- launches (each returns the launch error, cudaSuccess otherwise) ----
 
 // Step 1: kbar[b][j] for blocks_done[b] <= j < kv_len[b] / B; optionally records
@@ -94,8 +113,11 @@ bool score_tc_supported(const Dims &D, const Seqs &S);
 size_t score_tc_workspace(const Dims &D, const Seqs &S);
 // With scores_out set, writes each row's scores s[b][r][j] (j < n_c of the row) to
 // scores_out [batch][n_q][nb_cap] instead of selecting (sel is not touched).
+// pdl: the k̄ split and the scoring kernel are launched as programmatic dependents of
+// the kernel before them (qsa_forward's compression).
 cudaError_t launch_score_topk_tc(const Dims &D, const Seqs &S, const void *qi, const float *kbar, int32_t *sel,
-                                 void *scratch, int *status, cudaStream_t st, float *scores_out = nullptr);
+                                 void *scratch, int *status, cudaStream_t st, float *scores_out = nullptr,
+                                 bool pdl = false);
 
 // Steps 2 alone on CUDA cores (fp32): each row's scores s[b][r][j], j < n_c, into
 // scores [batch][n_q][nb_cap]; other entries are not written.
@@ -124,6 +146,11 @@ cudaError_t launch_proj_rope(const Dims &D, int hidden, float rope_theta, int rd
                              const void *w, const int32_t *pos0, int batch, int n_tok, void *q, void *qi, void *k,
                              void *v, void *ki, int kv_cap, int kv_row0, int *status, cudaStream_t st);
 
+// Checks every row of a selection list (ids in [0, n_c), strictly ascending, then -1
+// padding; padding rows all -1) and records QSA_ERR_DEVICE_CHECK on a violation.
+// Launched before the attention in the QSA_DEBUG build.
+cudaError_t launch_validate_sel(const Dims &D, const Seqs &S, const int32_t *sel, int *status, cudaStream_t st);
+
 // Step 4 on CUDA cores (fp32 accumulate), any supported shape.
 cudaError_t launch_attn_simt(const Dims &D, const Seqs &S, const void *q, const void *k,
                              const void *v, const int32_t *sel, void *out, int *status,
@@ -133,9 +160,10 @@ cudaError_t launch_attn_simt(const Dims &D, const Seqs &S, const void *q, const 
 // cudaErrorNotSupported when the shape is not served.
 bool attn_tc_supported(const Dims &D);
 size_t attn_tc_workspace(const Dims &D, const Seqs &S);
+// pdl: launched as a programmatic dependent of the kernel before it (qsa_forward's scoring).
 cudaError_t launch_attn_tc(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
                            const int32_t *sel, void *out, void *scratch, size_t scratch_bytes,
-                           int *status, cudaStream_t st);
+                           int *status, cudaStream_t st, bool pdl = false);
 
 // Step 4 on tcgen05 tensor cores, one 128-row tile per CTA with double-buffered S
 // (bf16, d = 256, G divides 128, block size a multiple of 64); no scratch.

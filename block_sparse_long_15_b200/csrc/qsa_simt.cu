@@ -7,6 +7,7 @@
 #include <math.h>
 
 #include "qsa_internal.h"
+#include "qsa_rowselect.cuh"
 
 namespace qsa {
 namespace {
@@ -22,11 +23,6 @@ __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
   return x;
-}
-__device__ __forceinline__ unsigned lanemask_lt() {
-  unsigned m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
 }
 
 // ---------------------------------------------------------------------------
@@ -55,6 +51,9 @@ k_compress(Dims D, Seqs S, const T *__restrict__ ki, const int32_t *__restrict__
            float *__restrict__ kbar, int32_t *__restrict__ blocks_out, int *status) {
   typedef typename Pair<T>::type P2;
   constexpr int kRows = sizeof(T) == 2 ? 64 : 32;  // rows loaded before they are summed
+  // a programmatic dependent (qsa_forward's next stage) may start its prologue now;
+  // it waits for this grid before it reads k̄
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (!seq_ok(S, b, status)) return;
@@ -187,7 +186,6 @@ __global__ void k_score_topk_simt(Dims D, Seqs S, const T *__restrict__ qi,
 // with block-wide counts; selected ids are written in ascending order.
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 512;
-constexpr int kMaxHi = 8;  // indexer heads scored together per k̄ piece
 
 // Decode prologue for sequence b, run by one CTA: append the new token at L-1
 // and, if that completes block j = L/B - 1, compress it and advance kbar_blocks.
@@ -295,68 +293,50 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
     return;
   }
   __syncthreads();
-  for (int j = tid; j < n_c; j += kRowThreads) {
-    const float4 *kr = (const float4 *)(j == j_new ? kbar_new : kb + (size_t)j * D.di);
-    float s = 0.f;
-    if (D.di <= 64) {
-      // the candidate's k̄ row in registers; the query heads, up to kMaxHi at a
-      // time, reuse it
-      float4 kv[16];
+  // Scores, eight lanes per candidate and four candidates per warp at a time: lane p
+  // of a candidate's eight holds dims 8p .. 8p + 7 of every 64-dim piece of the k̄ row,
+  // so one warp load reads four whole rows; each head's partial dots are summed
+  // across the eight lanes (three butterfly steps), then max(0, .) per head, summed.
+  {
+    const int slot = lane >> 3, part = lane & 7;
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = warp * 4; j0 < n_c; j0 += (kRowThreads / 32) * 4) {
+      const int j = j0 + slot;
+      const bool have = j < n_c;
+      const float *kr = (j == j_new) ? kbar_new : kb + (size_t)(have ? j : 0) * D.di;
+      float s = 0.f;
+      for (int h0 = 0; h0 < D.Hi; h0 += 4) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c0 = part * 8; c0 < D.di; c0 += 64) {
+          const float4 k0 = have ? *(const float4 *)(kr + c0) : zero4;
+          const float4 k1 = have ? *(const float4 *)(kr + c0 + 4) : zero4;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) kv[c] = (c < D.di / 4) ? kr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int h0 = 0; h0 < D.Hi; h0 += kMaxHi) {
-        float dot[kMaxHi];
-#pragma unroll
-        for (int h = 0; h < kMaxHi; ++h) dot[h] = 0.f;
-#pragma unroll
-        for (int h = 0; h < kMaxHi; ++h) {
-          if (h0 + h >= D.Hi) break;
-          const float4 *qh = (const float4 *)(qi_s + (h0 + h) * D.di);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            if (c >= D.di / 4) break;
-            const float4 a = qh[c];
-            dot[h] = fmaf(a.x, kv[c].x, dot[h]);
-            dot[h] = fmaf(a.y, kv[c].y, dot[h]);
-            dot[h] = fmaf(a.z, kv[c].z, dot[h]);
-            dot[h] = fmaf(a.w, kv[c].w, dot[h]);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < kMaxHi; ++h)
-          if (h0 + h < D.Hi) s += dot[h] > 0.f ? dot[h] : 0.f;
-      }
-    } else {
-      // wider rows in 64-float pieces whose 16 loads are all in flight together
-      for (int h0 = 0; h0 < D.Hi; h0 += kMaxHi) {
-        float dot[kMaxHi];
-#pragma unroll
-        for (int h = 0; h < kMaxHi; ++h) dot[h] = 0.f;
-        for (int c0 = 0; c0 < D.di / 4; c0 += 16) {
-          float4 kv[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) kv[c] = (c0 + c < D.di / 4) ? kr[c0 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int h = 0; h < kMaxHi; ++h) {
+          for (int h = 0; h < 4; ++h) {
             if (h0 + h >= D.Hi) break;
-            const float4 *qh = (const float4 *)(qi_s + (h0 + h) * D.di) + c0;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              if (c0 + c >= D.di / 4) break;
-              const float4 a = qh[c];
-              dot[h] = fmaf(a.x, kv[c].x, dot[h]);
-              dot[h] = fmaf(a.y, kv[c].y, dot[h]);
-              dot[h] = fmaf(a.z, kv[c].z, dot[h]);
-              dot[h] = fmaf(a.w, kv[c].w, dot[h]);
-            }
+            const float4 q0 = *(const float4 *)(qi_s + (h0 + h) * D.di + c0);
+            const float4 q1 = *(const float4 *)(qi_s + (h0 + h) * D.di + c0 + 4);
+            float a = acc[h];
+            a = fmaf(q0.x, k0.x, a);
+            a = fmaf(q0.y, k0.y, a);
+            a = fmaf(q0.z, k0.z, a);
+            a = fmaf(q0.w, k0.w, a);
+            a = fmaf(q1.x, k1.x, a);
+            a = fmaf(q1.y, k1.y, a);
+            a = fmaf(q1.z, k1.z, a);
+            a = fmaf(q1.w, k1.w, a);
+            acc[h] = a;
           }
         }
 #pragma unroll
-        for (int h = 0; h < kMaxHi; ++h)
-          if (h0 + h < D.Hi) s += dot[h] > 0.f ? dot[h] : 0.f;
+        for (int h = 0; h < 4; ++h) {
+          acc[h] += __shfl_xor_sync(kFull, acc[h], 1);
+          acc[h] += __shfl_xor_sync(kFull, acc[h], 2);
+          acc[h] += __shfl_xor_sync(kFull, acc[h], 4);
+          if (h0 + h < D.Hi) s += acc[h] > 0.f ? acc[h] : 0.f;
+        }
       }
+      if (have && part == 0) keys[j] = __float_as_uint(s);
     }
-    keys[j] = __float_as_uint(s);
   }
   __syncthreads();
   // Radix select of the k-th largest key, 8 bits at a time from the top: count the

@@ -15,7 +15,9 @@ from typing import Dict, Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libqsa.so")
+# QSA_LIBRARY may name another in-tree build of the library (libqsa_debug.so: the
+# same entry points with device-side checks of every selection list read).
+LIB_PATH = os.path.join(_PKG, os.environ.get("QSA_LIBRARY", "libqsa.so"))
 
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_CUDA, QSA_ERR_TIMEOUT, QSA_ERR_DEVICE_CHECK = range(6)
 QSA_DTYPE_BF16, QSA_DTYPE_FP32 = 0, 1
