@@ -10,6 +10,8 @@ steps. Also measured:
   workloads -- the same step on the long 64K prefill (planted blocks, top-k 64) and
                on the 8K prefill (16 / 2 heads, block 64, top-k 32), each with its
                attention kernel's roofline;
+  projection -- the projections + RoPE (qsa_project) over the headline batch's rows at
+               hidden size 2048, with cuBLAS's time for the bare GEMM as context;
   e2e       -- the headline step through qsa_forward with pinned HOST buffers, the
                host->device copy of the inputs (one copy from a pinned arena) and
                the device->host read of the output inside the timed region;
@@ -75,6 +77,7 @@ def parse_args(argv=None):
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-projection", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     p.add_argument("--batch", type=int, default=0,
                    help="override the headline workload's batch (a smaller case of the same shape, for "
@@ -378,8 +381,8 @@ def bench_prefill_e2e(args, w, inp, p, stream):
     two sets of device buffers, uploads on one stream, qsa_forward on another, downloads
     on a third, so that step i + 1's upload overlaps step i's compute and download
     (the host link is full duplex and the copy engines run beside the SMs). Every step
-    still uploads all of its inputs -- the packed arena, in four contiguous pieces on four
-    streams -- and reads its result back. Reported: throughput (ms per step over the pipelined run) and the
+    still uploads all of its inputs -- one copy of the packed arena -- and reads its
+    result back. Reported: throughput (ms per step over the pipelined run) and the
     latency of one step run alone."""
     import torch
 
@@ -398,13 +401,6 @@ def bench_prefill_e2e(args, w, inp, p, stream):
     h2d = arena.nbytes
     d2h = outs[0].numel() * outs[0].element_size()
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    # the arena's upload in N_UP contiguous pieces, each on a stream of its own, so that
-    # more than one copy engine drives the host link
-    N_UP = 4
-    piece = (arena.nbytes // N_UP) // (2 << 20) * (2 << 20) or arena.nbytes  # 2 MiB multiples
-    cuts = [min(arena.nbytes, i * piece) for i in range(N_UP + 1)]
-    cuts[-1] = arena.nbytes
-    s_up = [torch.cuda.Stream() for _ in range(N_UP)]
     free = [None, None]  # per buffer set: event after its last download
 
     def step(i):
@@ -412,15 +408,8 @@ def bench_prefill_e2e(args, w, inp, p, stream):
         x, o = sets[k], outs[k]
         if free[k] is not None:
             s_in.wait_event(free[k])
-        go = torch.cuda.Event()
-        go.record(s_in)
-        for j, su in enumerate(s_up):
-            if cuts[j + 1] <= cuts[j]:
-                continue
-            su.wait_event(go)
-            with torch.cuda.stream(su):
-                bufs[k][cuts[j]:cuts[j + 1]].copy_(arena.host[cuts[j]:cuts[j + 1]], non_blocking=True)
-            s_in.wait_stream(su)
+        with torch.cuda.stream(s_in):
+            bufs[k].copy_(arena.host, non_blocking=True)
         up = torch.cuda.Event()
         up.record(s_in)
         s_run.wait_event(up)
@@ -458,7 +447,71 @@ def bench_prefill_e2e(args, w, inp, p, stream):
         assert qsa.qsa_read_device_status(x.ws) == qsa.QSA_OK
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
     return dict(ms=a.elapsed_time(b) / n, h2d=h2d, d2h=d2h, latency_ms=statistics.median(lat),
-                copies_per_step={"h2d": sum(1 for j in range(N_UP) if cuts[j + 1] > cuts[j]), "d2h": 1})
+                copies_per_step={"h2d": 1, "d2h": 1})
+
+
+PROJ_HIDDEN = 2048  # Qwen4ExpTextConfig's hidden_size default
+
+
+def bench_projection(args, w, peaks, peak_src):
+    """The projection stage (qsa_project: q/k/v/indexer projections + RoPE, one tcgen05
+    GEMM) over every row of the workload's padded batch at hidden size 2048, weights and
+    hidden states synthetic (N(0,1) rows, N(0,1)/sqrt(hidden) weights, bf16), L2 flushed
+    between launches. cuBLAS's time for the same GEMM without the RoPE epilogue is
+    reported beside it as context."""
+    import torch
+
+    from block_sparse_long_15_b200 import qsa
+    dev = torch.cuda.current_device()
+    rows, hidden = w.batch * w.seq, PROJ_HIDDEN
+    n_out = w.Hq * w.d + 2 * w.Hkv * w.d + w.Hi * w.di + w.di
+    g = torch.Generator(device="cuda").manual_seed(7)
+    x = torch.randn(w.batch, w.seq, hidden, device="cuda", generator=g).to(torch.bfloat16)
+    wt = (torch.randn(n_out, hidden, device="cuda", generator=g) / hidden ** 0.5).to(torch.bfloat16)
+    bf = torch.bfloat16
+    q = torch.empty(w.batch, w.seq, w.Hq, w.d, dtype=bf, device="cuda")
+    qi = torch.empty(w.batch, w.seq, w.Hi, w.di, dtype=bf, device="cuda")
+    k = torch.empty(w.batch, w.Hkv, w.seq, w.d, dtype=bf, device="cuda")
+    v = torch.empty_like(k)
+    ki = torch.empty(w.batch, w.seq, w.di, dtype=bf, device="cuda")
+    q_first = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
+    cfg = qsa.config_for(w)
+    pc = qsa.qsa_proj_config_t(hidden, 1e6, w.d, w.di)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(dev, L2_FLUSH_BYTES)
+
+    def timed(fn, n):
+        out = []
+        for _ in range(n):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            out.append(a.elapsed_time(b))
+        return statistics.median(out)
+
+    run = lambda: qsa.qsa_project(cfg, pc, x, wt, q_first, q, qi, k, v, ki, 0, ws)
+    for _ in range(args.warmup):
+        run()
+    ms = timed(run, max(5, args.steps))
+    assert qsa.qsa_read_device_status(ws) == qsa.QSA_OK
+    y = torch.empty(rows, n_out, dtype=bf, device="cuda")
+    gemm = lambda: torch.matmul(x.view(rows, hidden), wt.t(), out=y)
+    for _ in range(args.warmup):
+        gemm()
+    ms_lib = timed(gemm, max(5, args.steps))
+    flops = 2.0 * rows * hidden * n_out
+    sustained = ms >= LONG_STEP_MS
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    ach = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "rows": rows, "hidden_size": hidden, "n_out": n_out, "ms": ms,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                         "peak_source": (f"bf16_tflops_sustained of {peak_src}" if sustained
+                                         else f"bf16_tflops (burst) of {peak_src}"),
+                         "flops_per_launch": flops},
+            "cublas_gemm_ms": ms_lib, "cublas_gemm_tflops": flops / (ms_lib * 1e-3) / 1e12}
 
 
 def decode_kernel_bytes(w, inp):
@@ -654,6 +707,9 @@ def main(argv=None):
         torch.cuda.empty_cache()
     if extra:
         out["workloads"] = extra
+    if not args.no_projection:
+        out["projection"] = bench_projection(args, w, peaks, peak_src)
+        torch.cuda.empty_cache()
     if not args.no_decode:
         wd = W.WORKLOADS[args.decode_workload]
         dec = bench_decode(args, wd, info, peaks)

@@ -1,6 +1,7 @@
-// The exact per-row top-k selection by one warp, shared by the tensor-core prefill
-// scoring kernel and the select-from-scores kernel, so that both take the same ids
-// from the same keys.
+// Per-row scoring and selection pieces: the fp32 score of one candidate block (the
+// decode selection kernel and the few-row scoring kernel), and the exact per-row
+// top-k by one warp (the tensor-core prefill scoring and the select-from-scores
+// kernel), so that every path that shares them takes the same ids from the same keys.
 // Definitions: Hugging Face Transformers model doc "Qwen4-Exp", intro paragraph on
 // QSA (multiple query heads score compressed key blocks, the most relevant blocks
 // are selected) and Qwen4ExpTextConfig indexer_budget.
@@ -14,6 +15,75 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
+}
+
+constexpr int kScoreMaxHi = 8;  // indexer heads scored together per k̄ piece
+
+// s_j = sum_h max(0, qi[h] . kbar_j) in fp32 for one candidate, computed by one thread:
+// qi_s [Hi][di] (fp32, any memory), kr the candidate's k̄ row (16-byte aligned,
+// di % 4 == 0). Dots run in dim order, four at a time from float4 pairs; heads are
+// summed in head order.
+__device__ __forceinline__ float block_score_fp32(const float *qi_s, int Hi, int di, const float4 *kr) {
+  float s = 0.f;
+  if (di <= 64) {
+    // the candidate's k̄ row in registers; the query heads, up to kScoreMaxHi at a
+    // time, reuse it
+    float4 kv[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) kv[c] = (c < di / 4) ? kr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int h0 = 0; h0 < Hi; h0 += kScoreMaxHi) {
+      float dot[kScoreMaxHi];
+#pragma unroll
+      for (int h = 0; h < kScoreMaxHi; ++h) dot[h] = 0.f;
+#pragma unroll
+      for (int h = 0; h < kScoreMaxHi; ++h) {
+        if (h0 + h >= Hi) break;
+        const float4 *qh = (const float4 *)(qi_s + (h0 + h) * di);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          if (c >= di / 4) break;
+          const float4 a = qh[c];
+          dot[h] = fmaf(a.x, kv[c].x, dot[h]);
+          dot[h] = fmaf(a.y, kv[c].y, dot[h]);
+          dot[h] = fmaf(a.z, kv[c].z, dot[h]);
+          dot[h] = fmaf(a.w, kv[c].w, dot[h]);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < kScoreMaxHi; ++h)
+        if (h0 + h < Hi) s += dot[h] > 0.f ? dot[h] : 0.f;
+    }
+  } else {
+    // wider rows in 64-float pieces whose 16 loads are all in flight together
+    for (int h0 = 0; h0 < Hi; h0 += kScoreMaxHi) {
+      float dot[kScoreMaxHi];
+#pragma unroll
+      for (int h = 0; h < kScoreMaxHi; ++h) dot[h] = 0.f;
+      for (int c0 = 0; c0 < di / 4; c0 += 16) {
+        float4 kv[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) kv[c] = (c0 + c < di / 4) ? kr[c0 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < kScoreMaxHi; ++h) {
+          if (h0 + h >= Hi) break;
+          const float4 *qh = (const float4 *)(qi_s + (h0 + h) * di) + c0;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            if (c0 + c >= di / 4) break;
+            const float4 a = qh[c];
+            dot[h] = fmaf(a.x, kv[c].x, dot[h]);
+            dot[h] = fmaf(a.y, kv[c].y, dot[h]);
+            dot[h] = fmaf(a.z, kv[c].z, dot[h]);
+            dot[h] = fmaf(a.w, kv[c].w, dot[h]);
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < kScoreMaxHi; ++h)
+        if (h0 + h < Hi) s += dot[h] > 0.f ? dot[h] : 0.f;
+    }
+  }
+  return s;
 }
 
 // Exact top-k of one row by a warp: writes out[0 .. k) with the ids of the k largest

@@ -293,50 +293,9 @@ k_score_topk_row(Dims D, Seqs S, const T *__restrict__ qi, const float *kbar, in
     return;
   }
   __syncthreads();
-  // Scores, eight lanes per candidate and four candidates per warp at a time: lane p
-  // of a candidate's eight holds dims 8p .. 8p + 7 of every 64-dim piece of the k̄ row,
-  // so one warp load reads four whole rows; each head's partial dots are summed
-  // across the eight lanes (three butterfly steps), then max(0, .) per head, summed.
-  {
-    const int slot = lane >> 3, part = lane & 7;
-    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = warp * 4; j0 < n_c; j0 += (kRowThreads / 32) * 4) {
-      const int j = j0 + slot;
-      const bool have = j < n_c;
-      const float *kr = (j == j_new) ? kbar_new : kb + (size_t)(have ? j : 0) * D.di;
-      float s = 0.f;
-      for (int h0 = 0; h0 < D.Hi; h0 += 4) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int c0 = part * 8; c0 < D.di; c0 += 64) {
-          const float4 k0 = have ? *(const float4 *)(kr + c0) : zero4;
-          const float4 k1 = have ? *(const float4 *)(kr + c0 + 4) : zero4;
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            if (h0 + h >= D.Hi) break;
-            const float4 q0 = *(const float4 *)(qi_s + (h0 + h) * D.di + c0);
-            const float4 q1 = *(const float4 *)(qi_s + (h0 + h) * D.di + c0 + 4);
-            float a = acc[h];
-            a = fmaf(q0.x, k0.x, a);
-            a = fmaf(q0.y, k0.y, a);
-            a = fmaf(q0.z, k0.z, a);
-            a = fmaf(q0.w, k0.w, a);
-            a = fmaf(q1.x, k1.x, a);
-            a = fmaf(q1.y, k1.y, a);
-            a = fmaf(q1.z, k1.z, a);
-            a = fmaf(q1.w, k1.w, a);
-            acc[h] = a;
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          acc[h] += __shfl_xor_sync(kFull, acc[h], 1);
-          acc[h] += __shfl_xor_sync(kFull, acc[h], 2);
-          acc[h] += __shfl_xor_sync(kFull, acc[h], 4);
-          if (h0 + h < D.Hi) s += acc[h] > 0.f ? acc[h] : 0.f;
-        }
-      }
-      if (have && part == 0) keys[j] = __float_as_uint(s);
-    }
+  for (int j = tid; j < n_c; j += kRowThreads) {
+    const float4 *kr = (const float4 *)(j == j_new ? kbar_new : kb + (size_t)j * D.di);
+    keys[j] = __float_as_uint(block_score_fp32(qi_s, D.Hi, D.di, kr));
   }
   __syncthreads();
   // Radix select of the k-th largest key, 8 bits at a time from the top: count the
