@@ -17,7 +17,8 @@ steps. Also measured:
                the device->host read of the output inside the timed region;
   decode    -- one decode step for 64 sequences with caches of 4096..32768 tokens
                (CUDA-graph replay, L2 flushed between steps), plus its attention
-               kernel against the HBM roofline;
+               kernel against the HBM roofline; the same at head_dim 256, and the
+               step with the K/V cache offloaded to host memory;
   roofline  -- the attention kernel's selected-token FLOPs over its CUDA-event time
                against the measured bf16 tensor-core peak;
   cpu_baseline -- the fp64 CPU oracle on a bounded random sample of query rows.
@@ -71,9 +72,12 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="bf16_prefill_varlen_b8_s16384_leftpad")
-    p.add_argument("--extra-workloads", default="bf16_prefill_s65536_planted,bf16_prefill_s8192",
+    p.add_argument("--extra-workloads", default="bf16_prefill_s65536_planted,bf16_prefill_s8192,bf16_prefill_s8192_hd256",
                    help="comma-separated prefill workloads measured beside the headline ('' for none)")
     p.add_argument("--decode-workload", default="bf16_decode_b64_l4k_32k")
+    p.add_argument("--more-decode-workloads", default="bf16_decode_b64_l4k_32k_hd256",
+                   help="comma-separated decode workloads measured beside the main one ('' for none)")
+    p.add_argument("--no-offload", action="store_true", help="skip the offloaded decode step")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -537,12 +541,43 @@ def decode_step_bytes(w, inp):
     return total
 
 
-def bench_decode(args, wd, dist_info, peaks):
+def bench_decode_offload(args, wd, inp, peaks):
+    """The decode step with the attention K/V cache in page-locked host memory
+    (qsa_decode_offload): selection on the device, then only the attended blocks cross
+    the host link into a device staging cache. Median of a few steps, L2 flushed."""
+    import torch
+
+    from block_sparse_long_15_b200 import qsa
+    from block_sparse_long_15_b200.runner import QSADecodeOffload
+    d = QSADecodeOffload(wd, inp)
+    flush = L2Flush(torch.cuda.current_device(), L2_FLUSH_BYTES)
+    for _ in range(max(2, args.warmup)):
+        d()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(max(5, args.steps)):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        d()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    assert d.status() == qsa.QSA_OK
+    kb = decode_kernel_bytes(wd, inp)
+    ms = statistics.median(ts)
+    return {"workload": wd.name, "ms_per_step": ms, "host_link_bytes_per_step": kb,
+            "host_link_gbs": kb / (ms * 1e-3) / 1e9,
+            "note": "K/V cache in page-locked host memory; the attended blocks cross the host link each step"}
+
+
+def bench_decode(args, wd, dist_info, peaks, inp=None):
     import torch
 
     from block_sparse_long_15_b200 import qsa, workloads as W
     from block_sparse_long_15_b200.runner import QSADecode
-    inp = W.make_inputs(wd)
+    if inp is None:
+        inp = W.make_inputs(wd)
     d = QSADecode(wd, inp)
     dev = torch.cuda.current_device()
     flush = L2Flush(dev, L2_FLUSH_BYTES)
@@ -712,9 +747,21 @@ def main(argv=None):
         torch.cuda.empty_cache()
     if not args.no_decode:
         wd = W.WORKLOADS[args.decode_workload]
-        dec = bench_decode(args, wd, info, peaks)
+        dinp = W.make_inputs(wd)
+        dec = bench_decode(args, wd, info, peaks, dinp)
         dec["us_per_step"] = max_over_ranks(dec["us_per_step"], info)
         out["decode"] = dec
+        more = {}
+        for name in [x for x in args.more_decode_workloads.split(",") if x]:
+            dm = bench_decode(args, W.WORKLOADS[name], info, peaks)
+            dm["us_per_step"] = max_over_ranks(dm["us_per_step"], info)
+            more[name] = dm
+            torch.cuda.empty_cache()
+        if more:
+            out["decode_more"] = more
+        if not args.no_offload and info is None:  # single-GPU runs: it pins a 2 GB host cache
+            out["decode_offload"] = bench_decode_offload(args, wd, dinp, peaks)
+            torch.cuda.empty_cache()
     if cpu_inp is not None:
         out["cpu_baseline"] = cpu_oracle_rate(w, cpu_inp, args.cpu_seconds)
     if rank == 0:

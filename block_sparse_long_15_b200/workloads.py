@@ -64,7 +64,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads of the benchmark description, by what they are.
+# The five workloads of the benchmark description, by what they are, and two at head_dim 256.
 WORKLOADS: Dict[str, Workload] = {
     "tiny_fp32_prefill_s256": Workload(
         name="tiny_fp32_prefill_s256", mode="prefill", batch=1, seq=256, Hq=4, Hkv=1,
@@ -84,6 +84,15 @@ WORKLOADS: Dict[str, Workload] = {
         name="bf16_prefill_varlen_b8_s16384_leftpad", mode="prefill", batch=8,
         seq=16384, Hq=32, Hkv=4, d=128, Hi=8, di=64, block=128, topk=16, dtype="bf16",
         seed=4, std=0.5, pad_max=2048),
+    # the 8K prefill and the 64-sequence decode at head_dim 256, Qwen4ExpTextConfig's
+    # default head width
+    "bf16_prefill_s8192_hd256": Workload(
+        name="bf16_prefill_s8192_hd256", mode="prefill", batch=1, seq=8192, Hq=16, Hkv=2,
+        d=256, Hi=4, di=64, block=64, topk=32, dtype="bf16", seed=1, std=0.5),
+    "bf16_decode_b64_l4k_32k_hd256": Workload(
+        name="bf16_decode_b64_l4k_32k_hd256", mode="decode", batch=64, seq=32768, Hq=16,
+        Hkv=2, d=256, Hi=4, di=64, block=64, topk=32, dtype="bf16", seed=2, std=0.5,
+        len_min=4096, len_max=32768),
 }
 
 
