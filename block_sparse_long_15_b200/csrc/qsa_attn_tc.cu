@@ -11,7 +11,8 @@
 // (two 64-key halves; a half lies inside one block):
 //   warp 0      TMA producer: K and V chunks (128-byte swizzle) into two 2-deep
 //               rings, K released after its QK MMAs, V after its PV MMAs;
-//   warp 1      TMEM owner and single-thread MMA issuer. Tiles ping-pong: for
+//   warp 1      TMEM owner and MMA issuer (the warp runs the loop, one elected
+//               lane issues). Tiles ping-pong: for
 //               chunk i it issues O_A += P_A V_i, S_A = Q_A K_{i+1}^T, then the
 //               same for B, so one tile's softmax overlaps the other tile's MMAs.
 //               A tile with no row that sees a chunk skips it. MMAs run in issue
@@ -277,10 +278,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && has_work) {
+    // The whole warp runs the loop on warp-uniform values; one elected lane issues.
+    if (has_work) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, kChunk, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, kD, false, true);
-      bool fail = !mbar_wait(&bars[kBarQ], 0, kWaitNs);
+      bool fail = !warp_wait(&bars[kBarQ], 0);
       tc_fence_after();
       int n_pv0 = 0, n_pv1 = 0;  // PVs issued per tile
       // Shared-memory descriptors are built once; a k-step moves the start address,
@@ -297,54 +299,55 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t off_q = (uint64_t)(((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4);
           const uint64_t off_k = (uint64_t)(((kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32) >> 4);
-          mma_ss(d, qd + off_q, kd + off_k, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_ss_w(d, qd + off_q, kd + off_k, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[kBarSFull + w]);
+        mma_commit_w(&bars[kBarSFull + w]);
       };
       auto issue_pv = [&](int w, int i) -> bool {
         const int cnt = w ? n_pv1++ : n_pv0++;
-        if (!mbar_wait(&bars[kBarPFull + w], cnt & 1, kWaitNs)) return false;
+        if (!warp_wait(&bars[kBarPFull + w], cnt & 1)) return false;
         tc_fence_after();
         const uint64_t vd = v_desc0 + (uint64_t)(((i % kNV) * kKVBytes) >> 4);
         const uint32_t o = tbase + 256u + (uint32_t)(w * 128), pcol = tbase + (uint32_t)(w * 128);
         // keys 16 kk .. 16 kk + 15 of half kk / 4 sit at columns 64 (kk / 4) + 8 (kk % 4)
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(o, pcol + (kk >> 2) * 64 + (kk & 3) * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
-                 (cnt > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars[kBarPVDone + w]);
+          mma_ts_w(o, pcol + (kk >> 2) * 64 + (kk & 3) * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                   (cnt > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_w(&bars[kBarPVDone + w]);
         return true;
       };
       int c = next_chunk(bm0, bm1, nwords, 0);
       if (!fail && c >= 0) {
-        if (!mbar_wait(&bars[kBarKFull], 0, kWaitNs)) fail = true;
+        if (!warp_wait(&bars[kBarKFull], 0)) fail = true;
         tc_fence_after();
         for (int w = 0; w < kTiles && !fail; ++w)
           if (bit_of(w ? bm1 : bm0, c)) issue_qk(w, 0);
-        mma_commit(&bars[kBarKEmpty]);
+        mma_commit_w(&bars[kBarKEmpty]);
       }
       for (int i = 0; c >= 0 && !fail; ++i) {
         const int c1 = next_chunk(bm0, bm1, nwords, c + 1);
         // V of chunk i, with rows past the sequence end zeroed: their P is zero but
         // the buffer may hold anything there, and 0 * NaN is NaN.
-        if (!mbar_wait(&bars[kBarVFull + i % kNV], (i / kNV) & 1, kWaitNs)) { fail = true; break; }
+        if (!warp_wait(&bars[kBarVFull + i % kNV], (i / kNV) & 1)) { fail = true; break; }
         const int valid_rows = len - c * kChunk;
         if (valid_rows < kChunk && start + len < S.kv_cap) {
           uint8_t *vs = base + kOffV + (i % kNV) * kKVBytes;
-          for (int rr = max(valid_rows, 0); rr < kChunk; ++rr) {
+          for (int rr = max(valid_rows, 0) + lane; rr < kChunk; rr += 32) {
             uint4 *p0 = (uint4 *)(vs + rr * 128);
             uint4 *p1 = (uint4 *)(vs + kKVBytes / 2 + rr * 128);
 #pragma unroll
             for (int q = 0; q < 8; ++q) p0[q] = p1[q] = make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
+          __syncwarp();
         }
         bool k_ready = false;
         for (int w = 0; w < kTiles; ++w) {
           if (bit_of(w ? bm1 : bm0, c) && !issue_pv(w, i)) { fail = true; break; }
           if (c1 >= 0 && bit_of(w ? bm1 : bm0, c1)) {
             if (!k_ready) {
-              if (!mbar_wait(&bars[kBarKFull + (i + 1) % kNK], ((i + 1) / kNK) & 1, kWaitNs)) { fail = true; break; }
+              if (!warp_wait(&bars[kBarKFull + (i + 1) % kNK], ((i + 1) / kNK) & 1)) { fail = true; break; }
               tc_fence_after();
               k_ready = true;
             }
@@ -352,12 +355,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           }
         }
         if (fail) break;
-        mma_commit(&bars[kBarVEmpty + i % kNV]);
-        if (c1 >= 0) mma_commit(&bars[kBarKEmpty + (i + 1) % kNK]);
+        mma_commit_w(&bars[kBarVEmpty + i % kNV]);
+        if (c1 >= 0) mma_commit_w(&bars[kBarKEmpty + (i + 1) % kNK]);
         c = c1;
-        if (*abort_flag) fail = true;
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) fail = true;
       }
-      if (fail) {
+      if (fail && lane == 0) {
         record_status(P.status, QSA_ERR_TIMEOUT);
         *abort_flag = 1;
       }
