@@ -253,17 +253,18 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && has_work) {
+    // The whole warp runs the loop on warp-uniform values; one elected lane issues.
+    if (has_work) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, kCK, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, D_, false, true);
-      bool fail = !mbar_wait(&bars[kBarQ], 0, kWaitNs);
+      bool fail = !mbar_wait_warp(&bars[kBarQ], 0, kWaitNs);
       tc_fence_after();
       const uint64_t q_desc = sdesc_sw128(smem_u32(base + L::kOffQ), 16, 1024);
       const uint64_t k_desc0 = sdesc_sw128(smem_u32(base + L::kOffK), 16, 1024);
       const uint64_t v_desc0 = sdesc_sw128(smem_u32(base + L::kOffV), kCK * 128, 1024);
       // S(n) = Q K_n^T into S buffer n % 2; K is K-major, 64 keys x D_.
       auto issue_qk = [&](int n) -> bool {
-        if (!mbar_wait(&bars[kBarKFull + n % kNK], (n / kNK) & 1, kWaitNs)) return false;
+        if (!mbar_wait_warp(&bars[kBarKFull + n % kNK], (n / kNK) & 1, kWaitNs)) return false;
         tc_fence_after();
         const uint64_t kd = k_desc0 + (uint64_t)(((n % kNK) * L::kKVBytes) >> 4);
         const uint32_t d = tbase + (uint32_t)(D_ + (n & 1) * kCK);
@@ -271,10 +272,10 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         for (int kk = 0; kk < D_ / 16; ++kk) {
           const uint64_t off_q = (uint64_t)(((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4);
           const uint64_t off_k = (uint64_t)(((kk >> 2) * (kCK * 128) + (kk & 3) * 32) >> 4);
-          mma_ss(d, q_desc + off_q, kd + off_k, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_ss_w(d, q_desc + off_q, kd + off_k, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[kBarSFull + (n & 1)]);
-        mma_commit(&bars[kBarKEmpty + n % kNK]);
+        mma_commit_w(&bars[kBarSFull + (n & 1)]);
+        mma_commit_w(&bars[kBarKEmpty + n % kNK]);
         return true;
       };
       int n_total = 0;
@@ -283,34 +284,35 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       if (!fail && n_total > 1 && !issue_qk(1)) fail = true;
       int c = next_chunk(bm, nwords, 0);
       for (int n = 0; n < n_total && !fail; ++n, c = next_chunk(bm, nwords, c + 1)) {
-        if (!mbar_wait(&bars[kBarPFull + (n & 1)], (n >> 1) & 1, kWaitNs)) { fail = true; break; }
-        if (!mbar_wait(&bars[kBarVFull + n % kNV], (n / kNV) & 1, kWaitNs)) { fail = true; break; }
+        if (!mbar_wait_warp(&bars[kBarPFull + (n & 1)], (n >> 1) & 1, kWaitNs)) { fail = true; break; }
+        if (!mbar_wait_warp(&bars[kBarVFull + n % kNV], (n / kNV) & 1, kWaitNs)) { fail = true; break; }
         tc_fence_after();
         // V rows past the sequence end are zeroed: their P is zero but the buffer
         // may hold anything there, and 0 * NaN is NaN.
         const int valid_rows = len - c * kCK;
         if (valid_rows < kCK && start + len < S.kv_cap) {
           uint8_t *vs = base + L::kOffV + (n % kNV) * L::kKVBytes;
-          for (int rr = max(valid_rows, 0); rr < kCK; ++rr)
+          for (int rr = max(valid_rows, 0) + lane; rr < kCK; rr += 32)
             for (int q = 0; q < kGroups; ++q) {
               uint4 *p4 = (uint4 *)(vs + q * (kCK * 128) + rr * 128);
 #pragma unroll
               for (int e = 0; e < 8; ++e) p4[e] = make_uint4(0, 0, 0, 0);
             }
           fence_proxy_async_smem();
+          __syncwarp();
         }
         const uint64_t vd = v_desc0 + (uint64_t)(((n % kNV) * L::kKVBytes) >> 4);
         const uint32_t pcol = tbase + (uint32_t)(D_ + (n & 1) * kCK);
 #pragma unroll
         for (int kk = 0; kk < kCK / 16; ++kk)
-          mma_ts(tbase, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars[kBarVEmpty + n % kNV]);
-        mma_commit(&bars[kBarPVDone]);
+          mma_ts_w(tbase, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_w(&bars[kBarVEmpty + n % kNV]);
+        mma_commit_w(&bars[kBarPVDone]);
         // S(n + 2) goes into the buffer this PV has just read; MMAs run in issue order.
         if (n + 2 < n_total && !issue_qk(n + 2)) { fail = true; break; }
-        if (*abort_flag) fail = true;
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) fail = true;
       }
-      if (fail) {
+      if (fail && lane == 0) {
         record_status(P.status, QSA_ERR_TIMEOUT);
         *abort_flag = 1;
       }

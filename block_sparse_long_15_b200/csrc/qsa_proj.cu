@@ -163,32 +163,33 @@ k_proj_rope(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop on warp-uniform values; one elected lane issues.
+    {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, false, false);
       int it = 0, local = 0;
       bool fail = false;
       for (int tile = blockIdx.x; tile < n_tiles && !fail; tile += gridDim.x, ++local) {
         const int buf = local & 1;
         // the epilogue has drained this accumulator (its use two tiles ago)
-        if (local >= 2 && !mbar_wait(&acc_empty[buf], ((local >> 1) & 1) ^ 1, kWaitNs)) { fail = true; break; }
+        if (local >= 2 && !mbar_wait_warp(&acc_empty[buf], ((local >> 1) & 1) ^ 1, kWaitNs)) { fail = true; break; }
         tc_fence_after();
         const uint32_t d = tbase + (uint32_t)(buf * kBN);
         for (int ks = 0; ks < k_steps; ++ks, ++it) {
           const int st = it % kStages;
-          if (!mbar_wait(&full[st], (it / kStages) & 1, kWaitNs)) { fail = true; break; }
+          if (!mbar_wait_warp(&full[st], (it / kStages) & 1, kWaitNs)) { fail = true; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(base + st * kStageBytes), sb = sa + kABytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_ss(d, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024), idesc,
-                   (ks > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&empty[st]);
+            mma_ss_w(d, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024), idesc,
+                     (ks > 0 || kk > 0) ? 1u : 0u);
+          mma_commit_w(&empty[st]);
         }
         if (fail) break;
-        mma_commit(&acc_full[buf]);
-        if (*abort_flag) fail = true;
+        mma_commit_w(&acc_full[buf]);
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) fail = true;
       }
-      if (fail) {
+      if (fail && lane == 0) {
         record_status(P.status, QSA_ERR_TIMEOUT);
         *abort_flag = 1;
       }

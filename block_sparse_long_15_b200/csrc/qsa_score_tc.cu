@@ -136,15 +136,16 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && n_ct > 0) {
+    // The whole warp runs the loop on warp-uniform values; one elected lane issues.
+    if (n_ct > 0) {
       const uint32_t idesc = idesc_bf16_f32(kCand, N, false, false);
-      fail = !mbar_wait(&bars[0], 0, kWaitNs);
+      fail = !mbar_wait_warp(&bars[0], 0, kWaitNs);
       tc_fence_after();
       const uint32_t qa = smem_u32(qi_s);
       for (int ct = 0; ct < n_ct && !fail; ++ct) {
         const int st = ct & 1, buf = ct & 1;
-        if (ct >= 2 && !mbar_wait(&bars[7 + buf], ((ct >> 1) & 1) ^ 1, kWaitNs)) { fail = true; break; }
-        if (!mbar_wait(&bars[1 + st], (ct >> 1) & 1, kWaitNs)) { fail = true; break; }
+        if (ct >= 2 && !mbar_wait_warp(&bars[7 + buf], ((ct >> 1) & 1) ^ 1, kWaitNs)) { fail = true; break; }
+        if (!mbar_wait_warp(&bars[1 + st], (ct >> 1) & 1, kWaitNs)) { fail = true; break; }
         tc_fence_after();
         const uint32_t ka = smem_u32(kb_s + st * 2 * cand_bytes);
         const uint32_t d = tbase + (uint32_t)(buf * N);
@@ -153,10 +154,10 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
           for (int hf = 0; hf < halves; ++hf)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk, ++step)
-              mma_ss(d, sdesc_sw128(ka + part * cand_bytes + hf * (kCand * 128) + kk * 32, 16, 1024),
-                     sdesc_sw128(qa + hf * (N * 128) + kk * 32, 16, 1024), idesc, step > 0 ? 1u : 0u);
-        mma_commit(&bars[5 + buf]);
-        mma_commit(&bars[3 + st]);
+              mma_ss_w(d, sdesc_sw128(ka + part * cand_bytes + hf * (kCand * 128) + kk * 32, 16, 1024),
+                       sdesc_sw128(qa + hf * (N * 128) + kk * 32, 16, 1024), idesc, step > 0 ? 1u : 0u);
+        mma_commit_w(&bars[5 + buf]);
+        mma_commit_w(&bars[3 + st]);
       }
     }
   } else if (warp < 6) {
@@ -194,7 +195,7 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
       if (lane == 0) mbar_arrive(&bars[7 + buf]);
     }
   }
-  if (fail) record_status(P.status, QSA_ERR_TIMEOUT);
+  if (fail && lane == 0) record_status(P.status, QSA_ERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -216,6 +216,13 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                : "memory");
 }
 
+// A wait taken by a whole warp: the same result on every lane, so the warp stays
+// converged for the warp-collective calls that follow.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Warp-collective forms of the three calls above: every lane of the warp makes the
 // call with the same operands and elect.sync picks one lane to issue (the lowest
 // active one, so with the whole warp converged the same lane every time, which the
