@@ -18,16 +18,17 @@
 //               A tile with no row that sees a chunk skips it. MMAs run in issue
 //               order, which orders a QK after the PV that read the same columns;
 //   warps 2-9   softmax of tile A, warps 10-17 tile B. Warp w reads TMEM lanes
-//               32 (w % 4) .. and one 64-key half of the chunk, so every row has
-//               two softmax warps, one per half: tcgen05.ld of its 64 S columns,
-//               the row's mask for the half (a half of a selected block is
-//               visible whole, a trailing half up to the query position, anything
-//               else not at all), the half's row max, swapped with the partner
-//               warp through shared memory, online softmax with a lazily rescaled
-//               reference max that both halves compute alike, P (bf16) written
-//               over the half's first 32 S columns with tcgen05.st for the PV MMA
-//               (A operand from TMEM); each half rescales and writes out its 64
-//               columns of O, and the two partial row sums meet in the epilogue.
+//               32 (w % 4) + 16 s .. + 15 (s one bit of w) with 16x32bx2 accesses
+//               split 64 columns apart, so it owns 16 rows whole: thread t < 16 holds
+//               its row's first 64-key half of the chunk, thread t + 16 the second.
+//               Per chunk: tcgen05.ld of the half's 64 S columns, the row's mask for
+//               the half (a half of a selected block is visible whole, a trailing
+//               half up to the query position, anything else not at all), the
+//               half's max, the row max by one shuffle with the partner thread,
+//               online softmax with a lazily rescaled reference max, P (bf16)
+//               written over the half's first 32 S columns with tcgen05.st for the
+//               PV MMA (A operand from TMEM); each thread rescales and writes out
+//               its 64 columns of O, and the two partial row sums meet by a shuffle.
 // TMEM (512 columns): S of tile w at 128 w, O of tile w at 256 + 128 w; P of half
 // h of tile w at 128 w + 64 h.
 // Every wait is bounded; on expiry the kernel records QSA_ERR_TIMEOUT and unwinds.
@@ -50,7 +51,7 @@ constexpr int kChunk = 128;  // keys per chunk (MMA N of S = Q K^T, K of O += P 
 constexpr int kHalf = 64;    // mask granularity (smallest block size served)
 constexpr int kNK = 2;       // K ring depth
 constexpr int kNV = 2;       // V ring depth
-constexpr int kThreads = 576;  // producer, MMA, 2 tiles x 2 halves x 4 lane groups
+constexpr int kThreads = 576;  // producer, MMA, 2 tiles x 4 lane groups x 2 sixteen-row groups
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
@@ -62,9 +63,7 @@ constexpr uint32_t kOffK = kOffQ + kTiles * kQBytes;
 constexpr uint32_t kOffV = kOffK + kNK * kKVBytes;
 constexpr uint32_t kOffBar = kOffV + kNV * kKVBytes;
 constexpr uint32_t kOffMisc = kOffBar + 512;
-constexpr uint32_t kOffXch = kOffMisc + 64;          // [parity][tile][half][row] fp32
-constexpr uint32_t kXchBytes = 2 * kTiles * 2 * kRows * 4;
-constexpr uint32_t kOffSel = kOffXch + kXchBytes;
+constexpr uint32_t kOffSel = kOffMisc + 64;
 constexpr uint32_t kOffBitmap = kOffSel + kSelBytes;
 
 // barrier slots
@@ -76,8 +75,7 @@ constexpr int kBarVEmpty = kBarVFull + kNV;
 constexpr int kBarSFull = kBarVEmpty + kNV;  // [tile]
 constexpr int kBarPFull = kBarSFull + 2;     // [tile], 8 arrivals (one per softmax warp)
 constexpr int kBarPVDone = kBarPFull + 2;    // [tile]
-constexpr int kBarXch = kBarPVDone + 2;      // [tile][lane group], 2 arrivals (the two halves)
-constexpr int kNumBars = kBarXch + kTiles * 4;
+constexpr int kNumBars = kBarPVDone + 2;
 static_assert(kNumBars * 8 <= 512, "barrier area");
 
 struct TcParams {
@@ -190,7 +188,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i)
-      mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 8u : i >= kBarXch ? 2u : 1u);
+      mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 8u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -367,34 +365,26 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
+    // Warp (tile w, lane group q, sub-group s) owns rows 32 q + 16 s .. + 15 of tile w,
+    // whole: thread t < 16 holds row 32 q + 16 s + t's first 64-key half of every
+    // chunk (and the first 64 columns of its O), thread t + 16 the same row's second
+    // half (16x32bx2 TMEM accesses with a 64-column split).
     const int sw = warp - 2;
-    const int w = sw >> 3;         // tile
-    const int hh = (sw >> 2) & 1;  // this warp's 64-key half of every chunk, and 64 columns of O
-    const int lg = warp & 3;       // TMEM lane group
+    const int w = sw >> 3;          // tile
+    const int sub = (sw >> 2) & 1;  // which 16 of the lane group's 32 rows
+    const int lg = warp & 3;        // TMEM lane group
+    const int hh = lane >> 4;       // this thread's 64-key half of every chunk, and 64 columns of O
     const uint32_t *bm = w ? bm1 : bm0;
-    const int row = 32 * lg + lane;
+    const int row = 32 * lg + 16 * sub + (lane & 15);
     const int tok = w * T + row / G, h = row % G;
     const int r = r0 + tok, t = qf + r;
     const bool valid = has_work && r < S.n_q && t >= 0 && t < len;
     const int n_c = valid ? (t + 1) / B : 0;
     const int32_t *srow = sel_cached ? sel_s + tok * k : P.sel + ((size_t)b * S.n_q + (valid ? r : 0)) * k;
-    const uint32_t lane_addr = tbase + ((uint32_t)(32 * lg) << 16);
-    const uint32_t s_col = lane_addr + (uint32_t)(w * 128 + hh * 64);
-    const uint32_t o_col = lane_addr + 256u + (uint32_t)(w * 128 + hh * 64);
+    const uint32_t lane_addr = tbase + ((uint32_t)(32 * lg + 16 * sub) << 16);
+    const uint32_t s_col = lane_addr + (uint32_t)(w * 128);        // this thread reads from + 64 hh
+    const uint32_t o_col = lane_addr + 256u + (uint32_t)(w * 128);  // likewise
     const float sl2 = D.scale * 1.4426950408889634f;
-    float *const xch = (float *)(base + kOffXch);
-    uint64_t *const xbar = &bars[kBarXch + w * 4 + lg];
-    // Exchange number e of a per-row value with the partner warp (same rows, other
-    // half). Slots alternate by parity: a warp can be at most one exchange ahead.
-    auto swap = [&](float v, int e, float &other) -> bool {
-      float *slot = xch + ((e & 1) * kTiles + w) * 2 * kRows;
-      slot[hh * kRows + row] = v;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xbar);
-      if (!warp_wait(xbar, e & 1)) return false;
-      other = slot[(hh ^ 1) * kRows + row];
-      return true;
-    };
     float m_ref = -INFINITY, l = 0.f;
     int ptr = 0, n = 0;
     bool fail = false;
@@ -415,19 +405,20 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           }
         }
         const bool z = __all_sync(0xffffffffu, lim == 0);
-        // Masking per key is needed only where a lane sees part of the half (its
-        // trailing block) or the half reaches past the sequence end (the cache may
-        // hold NaN there). Otherwise each lane sees all 64 keys or none: a lane that
-        // sees none takes +inf as its reference, so its p = 2^(s - inf) is 0.
-        const bool part = __any_sync(0xffffffffu, lim > 0 && lim < kHalf) || c * kChunk + hh * kHalf + kHalf > len;
+        // Masking per key is needed only where a thread sees part of its half (its
+        // row's trailing block) or the chunk reaches past the sequence end (the cache
+        // may hold NaN there). Otherwise each thread sees all 64 keys of its half or
+        // none: one that sees none takes +inf as its reference, so its p = 2^(s - inf)
+        // is 0.
+        const bool part = __any_sync(0xffffffffu, lim > 0 && lim < kHalf) || c * kChunk + kChunk > len;
         if (!warp_wait(&bars[kBarSFull + w], n & 1)) { fail = true; break; }
         tc_fence_after();
-        // pass 1: the half's row max over its visible keys
+        // pass 1: the half's max over its visible keys
         float hmax = -INFINITY;
         if (!z) {
           uint32_t sv0[32], sv1[32];
-          tmem_ld32(s_col, sv0);
-          tmem_ld32(s_col + 32, sv1);
+          tmem_ld32_pair64(s_col, sv0);
+          tmem_ld32_pair64(s_col + 32, sv1);
           tmem_ld_wait();
           if (part) {
             hmax = fmaxf(max_quarter<false>(sv0, lim), max_quarter<false>(sv1, lim - 32));
@@ -436,9 +427,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             hmax = lim ? mx : -INFINITY;
           }
         }
-        float omax = -INFINITY;
-        if (!swap(hmax, n, omax)) { fail = true; break; }
-        const float cmax = fmaxf(hmax, omax) * sl2;
+        // the row's max over both halves: the other half is in thread lane ^ 16
+        const float cmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, 16)) * sl2;
         bool rescale = false;
         float alpha = 1.f;
         if (cmax > -INFINITY) {  // the row sees a key in this chunk
@@ -450,40 +440,40 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             m_ref = cmax;
           }
         }
-        // pass 2: P (bf16 pairs) over the half's first 32 S columns, once all 64 are read
+        // pass 2: P (bf16 pairs) over each half's first 32 S columns, once all 64 are read
         float psum = 0.f;
         if (z) {
           uint32_t zk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) zk[e] = 0u;
-          tmem_st32(s_col, zk);
+          tmem_st32_pair64(s_col, zk);
         } else {
           const uint64_t scale2 = f2_splat(sl2);
           const uint64_t negm2 = f2_splat(part || lim ? -m_ref : -INFINITY);
           uint32_t sv0[32], sv1[32];
-          tmem_ld32(s_col, sv0);
+          tmem_ld32_pair64(s_col, sv0);
           tmem_ld_wait();
           psum = part ? p_quarter_regs<false>(sv0, lim, scale2, negm2) : p_quarter_regs<true>(sv0, 32, scale2, negm2);
-          tmem_ld32(s_col + 32, sv1);
+          tmem_ld32_pair64(s_col + 32, sv1);
           tmem_ld_wait();
           psum += part ? p_quarter_regs<false>(sv1, lim - 32, scale2, negm2)
                        : p_quarter_regs<true>(sv1, 32, scale2, negm2);
-          tmem_st32_lo(s_col, sv0, sv1);
+          tmem_st32_pair64_lo(s_col, sv0, sv1);
         }
         if (__any_sync(0xffffffffu, rescale)) {
-          // The reference max moved up: scale this half of the row's O (and its part
-          // of l) by alpha. O is stable once this tile's previous PV has completed,
-          // and the next PV waits for this warp's arrival below.
+          // The reference max moved up: scale this thread's half of the row's O (and
+          // its part of l) by alpha. O is stable once this tile's previous PV has
+          // completed, and the next PV waits for this warp's arrival below.
           if (n >= 1 && !warp_wait(&bars[kBarPVDone + w], (n - 1) & 1)) { fail = true; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int cb = 0; cb < 2; ++cb) {
             uint32_t ov[32];
-            tmem_ld32(o_col + cb * 32, ov);
+            tmem_ld32_pair64(o_col + cb * 32, ov);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
-            tmem_st32(o_col + cb * 32, ov);
+            tmem_st32_pair64(o_col + cb * 32, ov);
           }
           l *= alpha;
         }
@@ -496,9 +486,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         if (*abort_flag) { fail = true; break; }
       }
     }
-    // the two halves' partial sums of the row
-    float l_other = 0.f;
-    if (has_work && n > 0 && !fail && !swap(l, n, l_other)) fail = true;
+    // the row's sum over both halves
+    const float l_other = __shfl_xor_sync(0xffffffffu, l, 16);
     if (fail) {
       record_status(P.status, QSA_ERR_TIMEOUT);
       *abort_flag = 1;
@@ -527,7 +516,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         uint32_t ov[16];
-        tmem_ld16(o_col + cb * 16, ov);
+        tmem_ld16_pair64(o_col + cb * 16, ov);
         tmem_ld_wait();
         uint32_t pk[8];
 #pragma unroll
