@@ -417,8 +417,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         float hmax = -INFINITY;
         if (!z) {
           uint32_t sv0[32], sv1[32];
-          tmem_ld32_pair64(s_col, sv0);
-          tmem_ld32_pair64(s_col + 32, sv1);
+          tmem_ld32_split<64>(s_col, sv0);
+          tmem_ld32_split<64>(s_col + 32, sv1);
           tmem_ld_wait();
           if (part) {
             hmax = fmaxf(max_quarter<false>(sv0, lim), max_quarter<false>(sv1, lim - 32));
@@ -446,19 +446,19 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           uint32_t zk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) zk[e] = 0u;
-          tmem_st32_pair64(s_col, zk);
+          tmem_st32_split<64>(s_col, zk);
         } else {
           const uint64_t scale2 = f2_splat(sl2);
           const uint64_t negm2 = f2_splat(part || lim ? -m_ref : -INFINITY);
           uint32_t sv0[32], sv1[32];
-          tmem_ld32_pair64(s_col, sv0);
+          tmem_ld32_split<64>(s_col, sv0);
           tmem_ld_wait();
           psum = part ? p_quarter_regs<false>(sv0, lim, scale2, negm2) : p_quarter_regs<true>(sv0, 32, scale2, negm2);
-          tmem_ld32_pair64(s_col + 32, sv1);
+          tmem_ld32_split<64>(s_col + 32, sv1);
           tmem_ld_wait();
           psum += part ? p_quarter_regs<false>(sv1, lim - 32, scale2, negm2)
                        : p_quarter_regs<true>(sv1, 32, scale2, negm2);
-          tmem_st32_pair64_lo(s_col, sv0, sv1);
+          tmem_st32_split_lo<64>(s_col, sv0, sv1);
         }
         if (__any_sync(0xffffffffu, rescale)) {
           // The reference max moved up: scale this thread's half of the row's O (and
@@ -469,11 +469,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll 1
           for (int cb = 0; cb < 2; ++cb) {
             uint32_t ov[32];
-            tmem_ld32_pair64(o_col + cb * 32, ov);
+            tmem_ld32_split<64>(o_col + cb * 32, ov);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
-            tmem_st32_pair64(o_col + cb * 32, ov);
+            tmem_st32_split<64>(o_col + cb * 32, ov);
           }
           l *= alpha;
         }
@@ -516,7 +516,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         uint32_t ov[16];
-        tmem_ld16_pair64(o_col + cb * 16, ov);
+        tmem_ld16_split<64>(o_col + cb * 16, ov);
         tmem_ld_wait();
         uint32_t pk[8];
 #pragma unroll

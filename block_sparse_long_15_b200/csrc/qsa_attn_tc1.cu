@@ -11,15 +11,19 @@
 // query position, or not at all):
 //   warp 0      TMA producer: K and V chunks (128-byte swizzle) into two 2-deep
 //               rings, K released after its QK MMA, V after its PV MMA;
-//   warp 1      TMEM owner and single-thread MMA issuer. S is double-buffered in
+//   warp 1      TMEM owner and MMA issuer (the warp runs the loop, one elected
+//               lane issues). S is double-buffered in
 //               TMEM: while the softmax works on chunk n, S of chunk n + 1 is
 //               already there, and the PV of chunk n is followed by the QK of chunk
 //               n + 2 into the buffer that PV has just read;
-//   warps 2-5   softmax, one warp per 32 rows (warp w reads TMEM lanes 32 (w % 4)
-//               ..), one thread per row: tcgen05.ld of the chunk's 64 logits, the
-//               row max, online softmax with a lazily rescaled reference max, P
+//   warps 2-9   softmax, 16 rows per warp, whole: warp w reads TMEM lanes
+//               32 (w % 4) + 16 s .. + 15 (s one bit of w) with 16x32bx2 accesses,
+//               so thread t < 16 holds its row's first 32 keys of the chunk and
+//               thread t + 16 the last 32: tcgen05.ld of the 32 logits, the row max by
+//               one shuffle, online softmax with a lazily rescaled reference max, P
 //               (bf16) over the first 32 columns of the S buffer for the PV MMA (A
-//               operand from TMEM); epilogue O / l rounded to bf16.
+//               operand from TMEM); each thread rescales and writes out half of the
+//               row's O; epilogue O / l rounded to bf16.
 // TMEM: O in columns [0, 256), S buffers at 256 and 320 (512 allocated); shared
 // memory about 200 KB, one CTA per SM. Served for head_dim 256 only: head_dim 128
 // takes the two-tile kernel (qsa_attn_tc.cu).
@@ -40,7 +44,7 @@ constexpr int kRows = 128;   // MMA M: (token, head) rows of the tile
 constexpr int kCK = 64;      // keys per chunk (MMA N of S = Q K^T, K of O += P V)
 constexpr int kNK = 2;       // K ring depth
 constexpr int kNV = 2;       // V ring depth
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA, 4 lane groups x 2 sixteen-row groups
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kSelBytes = 8192;  // selection lists of the unit, if they fit
 
@@ -51,7 +55,7 @@ constexpr int kBarKEmpty = kBarKFull + kNK;
 constexpr int kBarVFull = kBarKEmpty + kNK;
 constexpr int kBarVEmpty = kBarVFull + kNV;
 constexpr int kBarSFull = kBarVEmpty + kNV;  // [S buffer]
-constexpr int kBarPFull = kBarSFull + 2;     // [S buffer], 4 arrivals (one per softmax warp)
+constexpr int kBarPFull = kBarSFull + 2;     // [S buffer], 8 arrivals (one per softmax warp)
 constexpr int kBarPVDone = kBarPFull + 2;
 constexpr int kNumBars = kBarPVDone + 1;
 
@@ -176,7 +180,7 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   const bool sel_cached = T * k * 4 <= (int)kSelBytes;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 4u : 1u);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? 8u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -204,10 +208,11 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   // The tile's chunk set (selected blocks and trailing ranges of its tokens) and a
   // shared-memory copy of its selection lists.
   if (warp >= 2 && has_work) {
+    constexpr int kSoftThreads = kThreads - 64;
     const int ts = threadIdx.x - 64;
-    for (int w = ts; w < nwords; w += 128) bm[w] = 0;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    for (int e = ts; e < T * k; e += 128) {
+    for (int w = ts; w < nwords; w += kSoftThreads) bm[w] = 0;
+    asm volatile("bar.sync 1, %0;" ::"n"(kSoftThreads) : "memory");
+    for (int e = ts; e < T * k; e += kSoftThreads) {
       const int tok = e / k, i = e - tok * k, r = r0 + tok, t = qf + r;
       if (r >= S.n_q || t < 0 || t >= len) continue;
       const int j = P.sel[((size_t)b * S.n_q + r) * k + i];
@@ -215,7 +220,7 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       if (j < 0 || j >= (t + 1) / B) continue;
       for (int c = (j * B) / kCK; c <= (j * B + B - 1) / kCK; ++c) atomicOr(&bm[c >> 5], 1u << (c & 31));
     }
-    for (int tok = ts; tok < T; tok += 128) {
+    for (int tok = ts; tok < T; tok += kSoftThreads) {
       const int r = r0 + tok, t = qf + r;
       if (r >= S.n_q || t < 0 || t >= len) continue;
       const int lo = ((t + 1) / B) * B;
@@ -319,93 +324,100 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int row = 32 * (warp & 3) + lane;
+    // Warp (lane group q, sub-group s) owns rows 32 q + 16 s .. + 15, whole: thread
+    // t < 16 holds row 32 q + 16 s + t's first 32 keys of every chunk and the first
+    // D_/2 columns of its O, thread t + 16 the same row's last 32 keys and last D_/2
+    // columns (16x32bx2 TMEM accesses).
+    const int sw = warp - 2;
+    const int sub = sw >> 2;
+    const int lg = warp & 3;
+    const int hh = lane >> 4;
+    const int row = 32 * lg + 16 * sub + (lane & 15);
     const int tok = row / G, h = row % G;
     const int r = r0 + tok, t = qf + r;
     const bool valid = has_work && r < S.n_q && t >= 0 && t < len;
     const int n_c = valid ? (t + 1) / B : 0;
     const int32_t *srow = sel_cached ? sel_s + tok * k : P.sel + ((size_t)b * S.n_q + (valid ? r : 0)) * k;
-    const uint32_t lane_addr = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t lane_addr = tbase + ((uint32_t)(32 * lg + 16 * sub) << 16);
     const float sl2 = D.scale * 1.4426950408889634f;
     float m_ref = -INFINITY, l = 0.f;
     int ptr = 0, n = 0;
     bool fail = false;
     if (has_work) {
       for (int c = next_chunk(bm, nwords, 0); c >= 0; c = next_chunk(bm, nwords, c + 1), ++n) {
-        // keys of this chunk the row sees: a selected block's keys whole, the
+        // keys of this thread's 32 the row sees: a selected block's keys whole, the
         // trailing block's up to the query position, nothing otherwise
         int lim = 0;
         if (valid) {
-          const int key0 = c * kCK;
+          const int key0 = c * kCK + hh * 32;
           const int jb = key0 / B;
           if (jb < n_c) {
             while (ptr < k && srow[ptr] >= 0 && srow[ptr] < jb) ++ptr;
-            lim = (ptr < k && srow[ptr] == jb) ? kCK : 0;
+            lim = (ptr < k && srow[ptr] == jb) ? 32 : 0;
           } else {
             const int last = t - key0;
-            lim = last >= 0 ? min(last + 1, kCK) : 0;
+            lim = last >= 0 ? min(last + 1, 32) : 0;
           }
         }
         const bool z = __all_sync(0xffffffffu, lim == 0);
-        // Masking per key is needed only where a lane sees part of the chunk (its
-        // trailing block) or the chunk reaches past the sequence end (the cache may
-        // hold NaN there). Otherwise each lane sees all 64 keys or none: a lane that
+        // Masking per key is needed only where a thread sees part of its 32 keys (its
+        // row's trailing block) or the chunk reaches past the sequence end (the cache
+        // may hold NaN there). Otherwise each thread sees all its keys or none: one that
         // sees none takes +inf as its reference, so its p = 2^(s - inf) is 0.
-        const bool part = __any_sync(0xffffffffu, lim > 0 && lim < kCK) || c * kCK + kCK > len;
+        const bool part = __any_sync(0xffffffffu, lim > 0 && lim < 32) || c * kCK + kCK > len;
         const uint32_t s_col = lane_addr + (uint32_t)(D_ + (n & 1) * kCK);
         if (!warp_wait(&bars[kBarSFull + (n & 1)], (n >> 1) & 1)) { fail = true; break; }
         tc_fence_after();
         float psum = 0.f, alpha = 1.f;
         bool rescale = false;
-        if (z) {
-          uint32_t zk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) zk[e] = 0u;
-          tmem_st32(s_col, zk);
-        } else {
-          // the chunk's 64 logits stay in registers: row max, then P in place
-          uint32_t sv0[32], sv1[32];
-          tmem_ld32(s_col, sv0);
-          tmem_ld32(s_col + 32, sv1);
+        uint32_t sv[32];
+        float hmax = -INFINITY;
+        if (!z) {
+          // this thread's 32 logits stay in registers: max, then P in place
+          tmem_ld32_split<32>(s_col, sv);
           tmem_ld_wait();
-          float mx;
-          if (part) {
-            mx = fmaxf(max_quarter<false>(sv0, lim), max_quarter<false>(sv1, lim - 32));
-          } else {
-            mx = fmaxf(max_quarter<true>(sv0, 32), max_quarter<true>(sv1, 32));
-            if (!lim) mx = -INFINITY;
+          hmax = part ? max_quarter<false>(sv, lim) : (lim ? max_quarter<true>(sv, 32) : -INFINITY);
+        }
+        // the row max: the other 32 keys are in thread lane ^ 16
+        const float cmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, 16)) * sl2;
+        if (cmax > -INFINITY) {
+          if (m_ref == -INFINITY) {
+            m_ref = cmax;
+          } else if (cmax > m_ref + 8.f) {
+            rescale = true;
+            alpha = ex2_approx(m_ref - cmax);
+            m_ref = cmax;
           }
-          const float cmax = mx * sl2;
-          if (cmax > -INFINITY) {
-            if (m_ref == -INFINITY) {
-              m_ref = cmax;
-            } else if (cmax > m_ref + 8.f) {
-              rescale = true;
-              alpha = ex2_approx(m_ref - cmax);
-              m_ref = cmax;
-            }
-          }
+        }
+        uint32_t pk[16];
+        if (z) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
+        } else {
           const uint64_t scale2 = f2_splat(sl2);
           const uint64_t negm2 = f2_splat(part || lim ? -m_ref : -INFINITY);
-          psum = part ? p_quarter<false>(sv0, lim, scale2, negm2) + p_quarter<false>(sv1, lim - 32, scale2, negm2)
-                      : p_quarter<true>(sv0, 32, scale2, negm2) + p_quarter<true>(sv1, 32, scale2, negm2);
-          tmem_st32_lo(s_col, sv0, sv1);
+          psum = part ? p_quarter<false>(sv, lim, scale2, negm2) : p_quarter<true>(sv, 32, scale2, negm2);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = sv[e];
         }
+        // P of keys 32 hh .. 32 hh + 31 at columns 16 hh .. of the S buffer
+        tmem_st16_split<16>(s_col, pk);
         if (__any_sync(0xffffffffu, rescale)) {
-          // The reference max moved up: scale the row's O (and l) by alpha. O is
-          // stable once the previous chunk's PV has completed, and this chunk's PV
-          // waits for this warp's arrival below. S of this chunk being there proves
-          // the PV of chunk n - 2 complete, so one parity wait suffices.
+          // The reference max moved up: scale this thread's half of the row's O (and
+          // its part of l) by alpha. O is stable once the previous chunk's PV has
+          // completed, and this chunk's PV waits for this warp's arrival below. S of
+          // this chunk being there proves the PV of chunk n - 2 complete, so one
+          // parity wait suffices.
           if (n >= 1 && !warp_wait(&bars[kBarPVDone], (n - 1) & 1)) { fail = true; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int cb = 0; cb < D_ / 16; ++cb) {
-            uint32_t ov[16];
-            tmem_ld16(lane_addr + cb * 16, ov);
+          for (int cb = 0; cb < D_ / 64; ++cb) {
+            uint32_t ov[32];
+            tmem_ld32_split<D_ / 2>(lane_addr + cb * 32, ov);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
-            tmem_st16(lane_addr + cb * 16, ov);
+            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
+            tmem_st32_split<D_ / 2>(lane_addr + cb * 32, ov);
           }
           l *= alpha;
         }
@@ -417,6 +429,8 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (*abort_flag) { fail = true; break; }
       }
     }
+    // the row's sum over both key ranges
+    const float l_other = __shfl_xor_sync(0xffffffffu, l, 16);
     if (fail) {
       record_status(P.status, QSA_ERR_TIMEOUT);
       *abort_flag = 1;
@@ -435,22 +449,23 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
     tc_fence_after();
     const bool write = r < S.n_q && ok;
-    __nv_bfloat16 *orow = P.out + (((size_t)b * S.n_q + (write ? r : 0)) * D.Hq + g * G + h) * D_;
+    __nv_bfloat16 *orow = P.out + (((size_t)b * S.n_q + (write ? r : 0)) * D.Hq + g * G + h) * D_ + hh * (D_ / 2);
     // A row that is not a query of the sequence (left padding) may hold NaN queries,
     // hence NaN in O: its output is written as zeros by selection, not by scaling.
-    const bool keep = valid && l > 0.f;
-    const float inv = keep ? 1.f / l : 0.f;
+    const float lt = l + l_other;
+    const bool keep = valid && lt > 0.f;
+    const float inv = keep ? 1.f / lt : 0.f;
     if (__all_sync(0xffffffffu, !have_o)) {
       if (write) {
         uint4 *o4 = (uint4 *)orow;
 #pragma unroll 1
-        for (int q = 0; q < D_ / 8; ++q) o4[q] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < D_ / 16; ++q) o4[q] = make_uint4(0, 0, 0, 0);
       }
     } else {
 #pragma unroll 1
-      for (int cb = 0; cb < D_ / 16; ++cb) {
+      for (int cb = 0; cb < D_ / 32; ++cb) {
         uint32_t ov[16];
-        tmem_ld16(lane_addr + cb * 16, ov);
+        tmem_ld16_split<D_ / 2>(lane_addr + cb * 16, ov);
         tmem_ld_wait();
         uint32_t pk[8];
 #pragma unroll

@@ -148,38 +148,49 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 // 32 consecutive columns from the first 16 registers of each of two arrays: a[0 .. 15]
 // to columns 0 .. 15, b[0 .. 15] to columns 16 .. 31.
-// The same loads and stores in the 16x32bx2 shape with a 64-column half split: the
-// warp covers 16 lanes from the lane in taddr; threads 0-15 access lane (base + t) at
-// the columns from taddr, threads 16-31 lane (base + t - 16) at those columns + 64.
-// So a row's two 64-column halves sit in threads t and t + 16 of one warp.
-__device__ __forceinline__ void tmem_ld32_pair64(uint32_t taddr, uint32_t (&r)[32]) {
+// The same loads and stores in the 16x32bx2 shape with a half split of kSplit
+// columns: the warp covers 16 lanes from the lane in taddr; threads 0-15 access lane
+// (base + t) at the columns from taddr, threads 16-31 lane (base + t - 16) at those
+// columns + kSplit. So a row's two column ranges sit in threads t and t + 16 of one warp.
+template <int kSplit>
+__device__ __forceinline__ void tmem_ld32_split(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 64;"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
       : QSA_R8(0), QSA_R8(8), QSA_R8(16), QSA_R8(24)
-      : "r"(taddr));
+      : "r"(taddr), "n"(kSplit));
 }
-__device__ __forceinline__ void tmem_ld16_pair64(uint32_t taddr, uint32_t (&r)[16]) {
+template <int kSplit>
+__device__ __forceinline__ void tmem_ld16_split(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 64;"
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
       : QSA_R8(0), QSA_R8(8)
-      : "r"(taddr));
+      : "r"(taddr), "n"(kSplit));
 }
-__device__ __forceinline__ void tmem_st32_pair64(uint32_t taddr, const uint32_t (&r)[32]) {
+template <int kSplit>
+__device__ __forceinline__ void tmem_st32_split(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 64, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr), "n"(kSplit),
       QSA_W8(0), QSA_W8(8), QSA_W8(16), QSA_W8(24)
+      : "memory");
+}
+template <int kSplit>
+__device__ __forceinline__ void tmem_st16_split(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};"
+      ::"r"(taddr), "n"(kSplit), QSA_W8(0), QSA_W8(8)
       : "memory");
 }
 #define QSA_WB8(i) "r"(b[i]), "r"(b[i + 1]), "r"(b[i + 2]), "r"(b[i + 3]), "r"(b[i + 4]), "r"(b[i + 5]), \
                    "r"(b[i + 6]), "r"(b[i + 7])
 // 16x32bx2 store of a[0..15] then b[0..15] (32 columns per thread).
-__device__ __forceinline__ void tmem_st32_pair64_lo(uint32_t taddr, const uint32_t (&a)[32], const uint32_t (&b)[32]) {
+template <int kSplit>
+__device__ __forceinline__ void tmem_st32_split_lo(uint32_t taddr, const uint32_t (&a)[32], const uint32_t (&b)[32]) {
   const uint32_t(&r)[32] = a;
   asm volatile(
-      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 64, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr), "n"(kSplit),
       QSA_W8(0), QSA_W8(8), QSA_WB8(0), QSA_WB8(8)
       : "memory");
 }
