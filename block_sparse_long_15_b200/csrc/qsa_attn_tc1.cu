@@ -56,8 +56,9 @@ constexpr int kBarVFull = kBarKEmpty + kNK;
 constexpr int kBarVEmpty = kBarVFull + kNV;
 constexpr int kBarSFull = kBarVEmpty + kNV;  // [S buffer]
 constexpr int kBarPFull = kBarSFull + 2;     // [S buffer], 8 arrivals (one per softmax warp)
-constexpr int kBarPVDone = kBarPFull + 2;
-constexpr int kNumBars = kBarPVDone + 1;
+constexpr int kBarPVDone = kBarPFull + 2;    // one phase per PV
+constexpr int kBarODone = kBarPVDone + 1;    // once, after the last PV
+constexpr int kNumBars = kBarODone + 1;
 
 template <int D_>
 struct Layout {
@@ -317,6 +318,7 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (n + 2 < n_total && !issue_qk(n + 2)) { fail = true; break; }
         if (__any_sync(0xffffffffu, *abort_flag != 0)) fail = true;
       }
+      mma_commit_w(&bars[kBarODone]);
       if (fail && lane == 0) {
         record_status(P.status, QSA_ERR_TIMEOUT);
         *abort_flag = 1;
@@ -437,12 +439,10 @@ k_attn_tc1(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
     // ---------------------------------------------------------------- epilogue
     // All n PVs must be complete. Having seen S of chunk n - 1 only proves that the
-    // PV of chunk n - 3 is (it was issued before that QK), so the PV barrier may be
-    // two phases behind, and a parity wait cannot tell phase n from phase n - 2:
-    // wait for the last two phases in order.
-    bool have_o = has_work && n > 0 && !fail;
-    if (have_o && n >= 2) have_o = warp_wait(&bars[kBarPVDone], (n - 2) & 1);
-    if (have_o) have_o = warp_wait(&bars[kBarPVDone], (n - 1) & 1);
+    // PV of chunk n - 3 is, and by the time this warp waits the PV barrier may be
+    // anywhere from phase n - 2 to phase n, two of which share a parity; so the
+    // epilogue waits on a barrier committed once, after the last PV.
+    const bool have_o = has_work && n > 0 && !fail && warp_wait(&bars[kBarODone], 0);
     if (has_work && n > 0 && !fail && !have_o) {
       record_status(P.status, QSA_ERR_TIMEOUT);
       *abort_flag = 1;
