@@ -442,11 +442,46 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         }
         // pass 2: P (bf16 pairs) over each half's first 32 S columns, once all 64 are read
         float psum = 0.f;
+        // lanes L and L ^ 8 hold the same half of the warp's two tokens (every lane takes
+        // part in these shuffles, whatever branch it goes on to)
+        const int lim_x = __shfl_xor_sync(0xffffffffu, lim, 8);
+        const float m_x = __shfl_xor_sync(0xffffffffu, m_ref, 8);
+        const bool pairable = !part && __all_sync(0xffffffffu, !(lim > 0 && lim_x > 0));
         if (z) {
           uint32_t zk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) zk[e] = 0u;
           tmem_st32_split<64>(s_col, zk);
+        } else if (pairable) {
+          // Lanes L and L ^ 8 hold the same half of the warp's two tokens. When no such
+          // pair has both lanes seeing their half, the blind lane of a pair takes the
+          // seeing lane's keys 32..63 and computes them with that lane's reference:
+          // every lane then runs 32 exponentials instead of 64 (MUFU costs the same per
+          // warp instruction whatever the lanes that take part).
+          const bool mine = lim > 0, other = lim_x > 0;
+          const uint64_t scale2 = f2_splat(sl2);
+          const uint64_t negm2 = f2_splat(mine ? -m_ref : other ? -m_x : -INFINITY);
+          uint32_t sv0[32], sv1[32];
+          tmem_ld32_split<64>(s_col + 32, sv1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) sv1[u] = __shfl_xor_sync(0xffffffffu, sv1[u], 8);
+          tmem_ld32_split<64>(s_col, sv0);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) sv0[u] = mine ? sv0[u] : sv1[u];
+          const float ps = p_quarter_regs<true>(sv0, 32, scale2, negm2);
+          // the seeing lane's P of keys 32..63 and their sum, back from its partner
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const uint32_t back = __shfl_xor_sync(0xffffffffu, sv0[u], 8);
+            sv1[u] = mine ? back : 0u;
+          }
+          const float ps_other = __shfl_xor_sync(0xffffffffu, ps, 8);
+          psum = mine ? ps + ps_other : 0.f;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) sv0[u] = mine ? sv0[u] : 0u;
+          tmem_st32_split_lo<64>(s_col, sv0, sv1);
         } else {
           const uint64_t scale2 = f2_splat(sl2);
           const uint64_t negm2 = f2_splat(part || lim ? -m_ref : -INFINITY);
