@@ -9,8 +9,9 @@
 // share every K/V tile, and both tiles share every K/V chunk in shared memory.
 // The unit walks the union of its tokens' key sets in ascending 128-key chunks
 // (two 64-key halves; a half lies inside one block):
-//   warp 0      TMA producer: K and V chunks (128-byte swizzle) into two 2-deep
-//               rings, K released after its QK MMAs, V after its PV MMAs;
+//   warp 0      TMA producer: K and V chunks (128-byte swizzle) into a 2-deep ring
+//               whose entry j holds K of chunk j and V of chunk j - 1 under one
+//               barrier, released after the QK MMAs of chunk j;
 //   warp 1      TMEM owner and MMA issuer (the warp runs the loop, one elected
 //               lane issues). Tiles ping-pong: for
 //               chunk i it issues O_A += P_A V_i, S_A = Q_A K_{i+1}^T, then the
@@ -49,8 +50,7 @@ constexpr int kRows = 128;   // MMA M: (token, head) rows per tile
 constexpr int kTiles = 2;    // tiles per CTA sharing the K/V chunks
 constexpr int kChunk = 128;  // keys per chunk (MMA N of S = Q K^T, K of O += P V)
 constexpr int kHalf = 64;    // mask granularity (smallest block size served)
-constexpr int kNK = 2;       // K ring depth
-constexpr int kNV = 2;       // V ring depth
+constexpr int kNE = 2;       // ring depth: entry j holds K of chunk j and V of chunk j - 1
 constexpr int kThreads = 576;  // producer, MMA, 2 tiles x 4 lane groups x 2 sixteen-row groups
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -59,20 +59,18 @@ constexpr uint32_t kQBytes = kRows * kD * 2;    // 32 KB per tile, two 64-column
 constexpr uint32_t kKVBytes = kChunk * kD * 2;  // 32 KB per K (or V) chunk, two halves
 constexpr uint32_t kSelBytes = 16384;           // selection lists of the unit, if they fit
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTiles * kQBytes;
-constexpr uint32_t kOffV = kOffK + kNK * kKVBytes;
-constexpr uint32_t kOffBar = kOffV + kNV * kKVBytes;
+constexpr uint32_t kEntryBytes = 2 * kKVBytes;  // K at + 0, V at + kKVBytes
+constexpr uint32_t kOffE = kOffQ + kTiles * kQBytes;
+constexpr uint32_t kOffBar = kOffE + kNE * kEntryBytes;
 constexpr uint32_t kOffMisc = kOffBar + 512;
 constexpr uint32_t kOffSel = kOffMisc + 64;
 constexpr uint32_t kOffBitmap = kOffSel + kSelBytes;
 
 // barrier slots
 constexpr int kBarQ = 0;
-constexpr int kBarKFull = 1;
-constexpr int kBarKEmpty = kBarKFull + kNK;
-constexpr int kBarVFull = kBarKEmpty + kNK;
-constexpr int kBarVEmpty = kBarVFull + kNV;
-constexpr int kBarSFull = kBarVEmpty + kNV;  // [tile]
+constexpr int kBarFull = 1;                  // [ring entry]
+constexpr int kBarEmpty = kBarFull + kNE;    // [ring entry]
+constexpr int kBarSFull = kBarEmpty + kNE;   // [tile]
 constexpr int kBarPFull = kBarSFull + 2;     // [tile], 8 arrivals (one per softmax warp)
 constexpr int kBarPVDone = kBarPFull + 2;    // [tile]
 constexpr int kNumBars = kBarPVDone + 2;
@@ -247,30 +245,35 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // Ring entry j: K of union chunk j (if any) and V of chunk j - 1 (if any), one
+    // barrier for both, so the MMA warp takes one wait per chunk for PV(j - 1) and
+    // QK(j), which it issues together.
     if (lane == 0 && has_work) {
-      int i = 0;
-      for (int c = next_chunk(bm0, bm1, nwords, 0); c >= 0;
-           c = next_chunk(bm0, bm1, nwords, c + 1), ++i) {
-        const int y = start + c * kChunk, z = b * D.Hkv + g;
-        const int sk = i % kNK, sv = i % kNV;
-        if (i >= kNK && !mbar_wait(&bars[kBarKEmpty + sk], ((i / kNK) & 1) ^ 1, kWaitNs)) {
+      const int z = b * D.Hkv + g;
+      int j = 0, cp = -1;
+      int c = next_chunk(bm0, bm1, nwords, 0);
+      while (c >= 0 || cp >= 0) {
+        const int se = j % kNE;
+        if (j >= kNE && !mbar_wait(&bars[kBarEmpty + se], ((j / kNE) & 1) ^ 1, kWaitNs)) {
           record_status(P.status, QSA_ERR_TIMEOUT);
           *abort_flag = 1;
           break;
         }
-        uint8_t *ks = base + kOffK + sk * kKVBytes;
-        mbar_arrive_expect_tx(&bars[kBarKFull + sk], kKVBytes);
-        tma_load_3d(&tm_k, &bars[kBarKFull + sk], ks, 0, y, z);
-        tma_load_3d(&tm_k, &bars[kBarKFull + sk], ks + kKVBytes / 2, 64, y, z);
-        if (i >= kNV && !mbar_wait(&bars[kBarVEmpty + sv], ((i / kNV) & 1) ^ 1, kWaitNs)) {
-          record_status(P.status, QSA_ERR_TIMEOUT);
-          *abort_flag = 1;
-          break;
+        uint8_t *es = base + kOffE + se * kEntryBytes;
+        mbar_arrive_expect_tx(&bars[kBarFull + se], (c >= 0 ? kKVBytes : 0u) + (cp >= 0 ? kKVBytes : 0u));
+        if (c >= 0) {
+          const int y = start + c * kChunk;
+          tma_load_3d(&tm_k, &bars[kBarFull + se], es, 0, y, z);
+          tma_load_3d(&tm_k, &bars[kBarFull + se], es + kKVBytes / 2, 64, y, z);
         }
-        uint8_t *vs = base + kOffV + sv * kKVBytes;
-        mbar_arrive_expect_tx(&bars[kBarVFull + sv], kKVBytes);
-        tma_load_3d(&tm_v, &bars[kBarVFull + sv], vs, 0, y, z);
-        tma_load_3d(&tm_v, &bars[kBarVFull + sv], vs + kKVBytes / 2, 64, y, z);
+        if (cp >= 0) {
+          const int y = start + cp * kChunk;
+          tma_load_3d(&tm_v, &bars[kBarFull + se], es + kKVBytes, 0, y, z);
+          tma_load_3d(&tm_v, &bars[kBarFull + se], es + kKVBytes + kKVBytes / 2, 64, y, z);
+        }
+        cp = c;
+        c = c >= 0 ? next_chunk(bm0, bm1, nwords, c + 1) : -1;
+        ++j;
         if (*abort_flag) break;
       }
     }
@@ -287,11 +290,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       // which is the low field of the descriptor, so it is a 64-bit add of
       // (byte offset >> 4).
       const uint64_t q_desc0 = sdesc_sw128(smem_u32(base + kOffQ), 16, 1024);
-      const uint64_t k_desc0 = sdesc_sw128(smem_u32(base + kOffK), 16, 1024);
-      const uint64_t v_desc0 = sdesc_sw128(smem_u32(base + kOffV), kKVBytes / 2, 1024);
-      auto issue_qk = [&](int w, int i) {
+      const uint64_t k_desc0 = sdesc_sw128(smem_u32(base + kOffE), 16, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(smem_u32(base + kOffE + kKVBytes), kKVBytes / 2, 1024);
+      // S_w = Q_w K^T from ring entry se
+      auto issue_qk = [&](int w, int se) {
         const uint64_t qd = q_desc0 + (uint64_t)((w * kQBytes) >> 4);
-        const uint64_t kd = k_desc0 + (uint64_t)(((i % kNK) * kKVBytes) >> 4);
+        const uint64_t kd = k_desc0 + (uint64_t)((se * kEntryBytes) >> 4);
         const uint32_t d = tbase + (uint32_t)(w * 128);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -301,11 +305,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         }
         mma_commit_w(&bars[kBarSFull + w]);
       };
-      auto issue_pv = [&](int w, int i) -> bool {
+      // O_w += P_w V from ring entry se, once P_w is written
+      auto issue_pv = [&](int w, int se) -> bool {
         const int cnt = w ? n_pv1++ : n_pv0++;
         if (!warp_wait(&bars[kBarPFull + w], cnt & 1)) return false;
         tc_fence_after();
-        const uint64_t vd = v_desc0 + (uint64_t)(((i % kNV) * kKVBytes) >> 4);
+        const uint64_t vd = v_desc0 + (uint64_t)((se * kEntryBytes) >> 4);
         const uint32_t o = tbase + 256u + (uint32_t)(w * 128), pcol = tbase + (uint32_t)(w * 128);
         // keys 16 kk .. 16 kk + 15 of half kk / 4 sit at columns 64 (kk / 4) + 8 (kk % 4)
 #pragma unroll
@@ -317,20 +322,23 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       };
       int c = next_chunk(bm0, bm1, nwords, 0);
       if (!fail && c >= 0) {
-        if (!warp_wait(&bars[kBarKFull], 0)) fail = true;
+        if (!warp_wait(&bars[kBarFull], 0)) fail = true;
         tc_fence_after();
         for (int w = 0; w < kTiles && !fail; ++w)
           if (bit_of(w ? bm1 : bm0, c)) issue_qk(w, 0);
-        mma_commit_w(&bars[kBarKEmpty]);
+        mma_commit_w(&bars[kBarEmpty]);
       }
       for (int i = 0; c >= 0 && !fail; ++i) {
         const int c1 = next_chunk(bm0, bm1, nwords, c + 1);
-        // V of chunk i, with rows past the sequence end zeroed: their P is zero but
-        // the buffer may hold anything there, and 0 * NaN is NaN.
-        if (!warp_wait(&bars[kBarVFull + i % kNV], (i / kNV) & 1)) { fail = true; break; }
+        // entry i + 1: V of chunk i and, if there is one, K of chunk i + 1. V rows past
+        // the sequence end are zeroed: their P is zero but the buffer may hold
+        // anything there, and 0 * NaN is NaN.
+        const int e = i + 1, se = e % kNE;
+        if (!warp_wait(&bars[kBarFull + se], (e / kNE) & 1)) { fail = true; break; }
+        tc_fence_after();
         const int valid_rows = len - c * kChunk;
         if (valid_rows < kChunk && start + len < S.kv_cap) {
-          uint8_t *vs = base + kOffV + (i % kNV) * kKVBytes;
+          uint8_t *vs = base + kOffE + se * kEntryBytes + kKVBytes;
           for (int rr = max(valid_rows, 0) + lane; rr < kChunk; rr += 32) {
             uint4 *p0 = (uint4 *)(vs + rr * 128);
             uint4 *p1 = (uint4 *)(vs + kKVBytes / 2 + rr * 128);
@@ -340,21 +348,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           fence_proxy_async_smem();
           __syncwarp();
         }
-        bool k_ready = false;
         for (int w = 0; w < kTiles; ++w) {
-          if (bit_of(w ? bm1 : bm0, c) && !issue_pv(w, i)) { fail = true; break; }
-          if (c1 >= 0 && bit_of(w ? bm1 : bm0, c1)) {
-            if (!k_ready) {
-              if (!warp_wait(&bars[kBarKFull + (i + 1) % kNK], ((i + 1) / kNK) & 1)) { fail = true; break; }
-              tc_fence_after();
-              k_ready = true;
-            }
-            issue_qk(w, i + 1);
-          }
+          if (bit_of(w ? bm1 : bm0, c) && !issue_pv(w, se)) { fail = true; break; }
+          if (c1 >= 0 && bit_of(w ? bm1 : bm0, c1)) issue_qk(w, se);
         }
         if (fail) break;
-        mma_commit_w(&bars[kBarVEmpty + i % kNV]);
-        if (c1 >= 0) mma_commit_w(&bars[kBarKEmpty + (i + 1) % kNK]);
+        mma_commit_w(&bars[kBarEmpty + se]);
         c = c1;
         if (__any_sync(0xffffffffu, *abort_flag != 0)) fail = true;
       }
