@@ -43,6 +43,8 @@ struct ScoreParams {
   int *status;
   int n_tiles;  // token tiles per sequence
   int N;        // kTok * Hi
+  int stages;   // candidate-tile stages and accumulator buffers: 1 when every token has at most
+                // kCand candidate blocks (one tile), else 2
 };
 
 // Split fp32 kbar into bf16 hi and lo planes [batch * nb_cap][di].
@@ -58,8 +60,10 @@ __global__ void k_kbar_split(const float *__restrict__ kbar, __nv_bfloat16 *__re
   }
 }
 
+// At most 64 registers a thread, so that two CTAs fit on an SM when the shared memory
+// and TMEM of one candidate stage allow it.
 template <int HI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant__ CUtensorMap tm_hi,
                 const __grid_constant__ CUtensorMap tm_lo, ScoreParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -72,8 +76,8 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
   const uint32_t qi_bytes = (uint32_t)N * di * 2;   // B operand: N rows (token, head)
   const uint32_t cand_bytes = (uint32_t)kCand * di * 2;
   uint8_t *qi_s = base;                             // [halves][N][128 B]
-  uint8_t *kb_s = base + qi_bytes;                  // [2 stages][hi, lo][halves][128][128 B]
-  uint64_t *bars = (uint64_t *)(kb_s + 4 * cand_bytes);
+  uint8_t *kb_s = base + qi_bytes;                  // [stages][hi, lo][halves][128][128 B]
+  uint64_t *bars = (uint64_t *)(kb_s + 2 * P.stages * cand_bytes);
   // bars: 0 q_full, 1..2 k_full[stage], 3..4 k_empty[stage], 5..6 d_full[buf], 7..8 d_empty[buf]
   uint32_t *tmem_slot = (uint32_t *)(bars + 16);
   int *ncs = (int *)(tmem_slot + 4);                // [kTok] candidates per token (-1: padding row)
@@ -96,8 +100,8 @@ k_score_topk_tc(const __grid_constant__ CUtensorMap tm_qi, const __grid_constant
     for (int i = 0; i < 9; ++i) mbar_init(&bars[i], (i >= 7) ? 4u : 1u);
     fence_mbar_init();
   }
-  // two accumulator buffers of N columns (a power of two >= 32)
-  const uint32_t tcols = (uint32_t)(2 * N < 32 ? 32 : 2 * N);
+  // P.stages accumulator buffers of N columns (a power of two >= 32)
+  const uint32_t tcols = (uint32_t)(P.stages * N < 32 ? 32 : P.stages * N);
   if (warp == 1) {
     tmem_alloc(tmem_slot, tcols);
     tmem_relinquish();
@@ -279,10 +283,11 @@ bool make_map2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
+int score_stages(int nb_tile_max) { return nb_tile_max <= kCand ? 1 : 2; }
 size_t smem_bytes(const Dims &D, int nb_tile_max) {
   const int N = kTok * D.Hi;
-  return 1024 + (size_t)N * D.di * 2 + 4 * (size_t)kCand * D.di * 2 + 16 * 8 + 16 + kTok * 4 +
-         (size_t)kTok * nb_tile_max * 4;
+  return 1024 + (size_t)N * D.di * 2 + 2 * (size_t)score_stages(nb_tile_max) * kCand * D.di * 2 + 16 * 8 + 16 +
+         kTok * 4 + (size_t)kTok * nb_tile_max * 4;
 }
 
 }  // namespace
@@ -325,6 +330,7 @@ cudaError_t launch_score_topk_tc(const Dims &D, const Seqs &S, const void *qi, c
   P.n_tiles = (S.n_q + kTok - 1) / kTok;
   P.N = kTok * D.Hi;
   const int nb_tiles = ((S.nb_cap + kCand - 1) / kCand) * kCand;
+  P.stages = score_stages(nb_tiles);
   const size_t smem = smem_bytes(D, nb_tiles);
   auto kern = D.Hi == 1 ? k_score_topk_tc<1> : D.Hi == 2 ? k_score_topk_tc<2> : D.Hi == 4 ? k_score_topk_tc<4>
                                                                                   : k_score_topk_tc<8>;
