@@ -177,7 +177,8 @@ qsa_status_t attn_dispatch(const Dims &D, const Seqs &S, const void *q, const vo
       return cuda_status(
           launch_attn_decode(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st, pdl));
     case kAttnTc:
-      return cuda_status(launch_attn_tc(D, S, q, k, v, sel, out, scratch, scratch_bytes, status_word(ws), st, pdl));
+      return cuda_status(
+          launch_attn_tc(D, S, q, k, v, sel, out, (unsigned *)((char *)ws + kSchedOffset), status_word(ws), st, pdl));
     case kAttnTc1:
       return cuda_status(launch_attn_tc1(D, S, q, k, v, sel, out, status_word(ws), st));
     default:

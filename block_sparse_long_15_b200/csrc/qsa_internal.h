@@ -25,8 +25,11 @@ struct Seqs {
   int nb_cap;  // kv_cap / B: rows of kbar per sequence
 };
 
-// Workspace layout: [0, 256) status word area, then kernel scratch.
+// Workspace layout: [0, 256) status word area, then kernel scratch. Within the status
+// area, the two words at kSchedOffset are the unit counters of the persistent prefill
+// attention kernel, which its last CTA sets back to zero.
 constexpr size_t kStatusBytes = 256;
+constexpr size_t kSchedOffset = 128;
 
 __device__ __forceinline__ void record_status(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
@@ -161,9 +164,10 @@ cudaError_t launch_attn_simt(const Dims &D, const Seqs &S, const void *q, const 
 bool attn_tc_supported(const Dims &D);
 size_t attn_tc_workspace(const Dims &D, const Seqs &S);
 // pdl: launched as a programmatic dependent of the kernel before it (qsa_forward's scoring).
+// sched: two zeroed words (unit ticket, CTAs done) the kernel leaves at zero.
 cudaError_t launch_attn_tc(const Dims &D, const Seqs &S, const void *q, const void *k, const void *v,
-                           const int32_t *sel, void *out, void *scratch, size_t scratch_bytes,
-                           int *status, cudaStream_t st, bool pdl = false);
+                           const int32_t *sel, void *out, unsigned *sched, int *status, cudaStream_t st,
+                           bool pdl = false);
 
 // Step 4 on tcgen05 tensor cores, one 128-row tile per CTA with double-buffered S
 // (bf16, d = 256, G divides 128, block size a multiple of 64); no scratch.

@@ -130,7 +130,8 @@ const char *qsa_status_string(qsa_status_t status);
  * must be all zero before its first use; the library leaves the parts it relies on
  * at zero again after each call, except after a call whose device wait ran out
  * (status QSA_ERR_TIMEOUT): zero the workspace again before reusing it. Its first
- * 256 bytes hold the status word (qsa_read_device_status reads and clears it). One workspace must not serve two
+ * 256 bytes hold the status word (qsa_read_device_status reads and clears it) and the
+ * prefill attention's unit counters. One workspace must not serve two
  * calls that run concurrently. */
 qsa_status_t qsa_workspace_size(const qsa_config_t *cfg, int32_t mode, int32_t batch, int32_t n_q,
                                 int32_t kv_cap, size_t *bytes);
