@@ -1,0 +1,51 @@
+"""The persistent prefill attention kernel: its CTAs take units from a ticket counter kept
+in the workspace's status page, and the last CTA sets the counters back to zero. These
+tests check that every call leaves the workspace at zero (its contract) and that the
+dynamic assignment of units to CTAs does not change a single output bit."""
+import pytest
+import torch
+
+from block_sparse_long_15_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+WL = W.WORKLOADS
+
+
+def _status_page(ws):
+    return ws[:256].cpu()
+
+
+@pytest.mark.parametrize("name", ["bf16_prefill_s8192", "bf16_prefill_varlen_b8_s16384_leftpad"])
+def test_repeated_calls_bit_identical_and_workspace_zero(cuda_lib, name):
+    from block_sparse_long_15_b200.runner import QSAPrefill
+    w = WL[name]
+    p = QSAPrefill(w, W.make_inputs(w))
+    outs = []
+    for _ in range(3):
+        out, sel = p()
+        torch.cuda.synchronize()
+        # status word and the attention's unit counters: all zero after the call
+        assert torch.count_nonzero(_status_page(p.ws)) == 0
+        outs.append((out.clone(), sel.clone()))
+    for out, sel in outs[1:]:
+        assert torch.equal(sel, outs[0][1])
+        assert torch.equal(out, outs[0][0])
+
+
+def test_standalone_attention_shares_the_workspace(cuda_lib):
+    """qsa_sparse_attn on the workspace qsa_forward used: same output, counters back at zero."""
+    qsa = cuda_lib
+    from block_sparse_long_15_b200.runner import QSAPrefill
+    w = W.small_variant(WL["bf16_prefill_s8192"], seq=2112)
+    p = QSAPrefill(w, W.make_inputs(w))
+    out_f, _ = p()
+    out_f = out_f.clone()
+    t = p.t
+    out = torch.empty_like(t["q"])
+    for _ in range(2):
+        qsa.qsa_sparse_attn(p.cfg, t["q"], t["k_cache"], t["v_cache"], t["sel"], t["kv_start"], t["kv_len"],
+                            t["q_first"], out, p.ws)
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(_status_page(p.ws)) == 0
+        assert torch.equal(out, out_f)
