@@ -49,3 +49,26 @@ def test_standalone_attention_shares_the_workspace(cuda_lib):
         torch.cuda.synchronize()
         assert torch.count_nonzero(_status_page(p.ws)) == 0
         assert torch.equal(out, out_f)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(seq=1100, Hq=2, Hkv=2, block=64, topk=12),   # G = 1: 256 tokens a unit, lists beyond the slot
+    dict(seq=1100, Hq=4, Hkv=2, block=64, topk=20),   # G = 2: lists beyond the slot, read from global
+    dict(seq=1100, Hq=8, Hkv=2, block=64, topk=5),    # G = 4: k not a multiple of 4
+    dict(seq=1100, Hq=16, Hkv=2, block=192, topk=3),  # a block size that is not a power of two
+    dict(seq=2200, Hq=16, Hkv=2, block=256, topk=4),  # a block of two chunks
+])
+def test_tc_attention_unit_shapes_full_rows(cuda_lib, shape):
+    """Unit shapes that take the builder's other paths (the lists loaded from global
+    memory, read entry by entry, blocks of several chunks): every row of a left-padded
+    batch against the oracle."""
+    import oracle
+    from tests.parity_util import compare
+    from tests.test_parity_gpu import assert_report, run_prefill
+    qsa = cuda_lib
+    w = W.small_variant(WL["bf16_prefill_varlen_b8_s16384_leftpad"], batch=2, pad_max=130, **shape)
+    assert qsa.qsa_attn_kernel_name(qsa.config_for(w)) == "tcgen05"
+    inp = W.make_inputs(w)
+    out, sel, _ = run_prefill(qsa, w, inp)
+    rep = compare(w, inp, out, sel, oracle.run(w, inp))
+    assert_report(rep, w)
