@@ -11,7 +11,9 @@
 // lies inside one block). The kernel is persistent: one CTA per SM takes units from
 // an atomic ticket, heaviest (latest) units first, and prepares the next unit while
 // the current one ends, so the selection read, the Q load and the first K chunk of
-// a unit overlap the previous unit's last chunks:
+// a unit overlap the previous unit's last chunks. The ticket and a count of CTAs
+// done with tickets sit in the workspace's status page; the last CTA sets both back
+// to zero, so the workspace is zero again after every call:
 //   warp 18     unit builder: takes the next ticket when the producer nears the end
 //               of the current unit, writes the unit's coordinates, its per-tile chunk
 //               bitmaps and a copy of its selection lists into one of two slots, and
@@ -27,6 +29,8 @@
 //               same for B, so one tile's softmax overlaps the other tile's MMAs.
 //               A tile with no row that sees a chunk skips it. MMAs run in issue
 //               order, which orders a QK after the PV that read the same columns;
+//               a tile's first PV of a unit overwrites O, after the softmax warps
+//               have read the previous unit's O (their P of the new unit comes later);
 //   warps 2-9   softmax of tile A, warps 10-17 tile B. Warp w reads TMEM lanes
 //               32 (w % 4) + 16 s .. + 15 (s one bit of w) with 16x32bx2 accesses
 //               split 64 columns apart, so it owns 16 rows whole: thread t < 16 holds
