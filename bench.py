@@ -257,9 +257,13 @@ def cpu_oracle_rate(w, inp, seconds, seed=0):
         oracle.run(w, inp, rows={b: sorted(v) for b, v in by_b.items()})
         return len(idx), time.perf_counter() - t0
 
-    n, dt = run(32)
-    per_row = dt / max(n, 1)
-    n_main = int(min(len(rows_all), max(32, seconds / max(per_row, 1e-6))))
+    # A call has a fixed part (the workload's block means, set-up) besides its per-row
+    # work: two pilot sizes separate them, so the main sample lasts about `seconds`.
+    n1, d1 = run(32)
+    n2, d2 = run(min(256, len(rows_all)))
+    per_row = max((d2 - d1) / max(n2 - n1, 1), d2 / max(n2, 1) / 16, 1e-6)
+    fixed = max(d1 - per_row * n1, 0.0)
+    n_main = int(min(len(rows_all), max(n2, (seconds - fixed) / per_row)))
     n, dt = run(n_main)
     return {"value": n / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
             "sample": f"{n} query rows drawn uniformly (seed {seed}) from the {len(rows_all)} real rows of "
