@@ -72,3 +72,27 @@ def test_tc_attention_unit_shapes_full_rows(cuda_lib, shape):
     out, sel, _ = run_prefill(qsa, w, inp)
     rep = compare(w, inp, out, sel, oracle.run(w, inp))
     assert_report(rep, w)
+
+
+@pytest.mark.parametrize("name,shape,calls", [
+    ("bf16_prefill_s8192", None, 200),
+    ("bf16_prefill_varlen_b8_s16384_leftpad", dict(seq=1100, Hq=2, Hkv=2, block=64, topk=12), 150),
+    ("bf16_prefill_varlen_b8_s16384_leftpad", dict(seq=2200, Hq=16, Hkv=2, block=256, topk=4), 150),
+])
+def test_soak_many_calls(cuda_lib, name, shape, calls):
+    """Many calls in a row on one workspace: the status word stays clear, every output
+    equals the first bit for bit, and the counters are back at zero at the end -- the
+    dynamic assignment of units to CTAs differs from call to call."""
+    from block_sparse_long_15_b200.runner import QSAPrefill
+    w = WL[name] if shape is None else W.small_variant(WL[name], batch=2, pad_max=130, **shape)
+    p = QSAPrefill(w, W.make_inputs(w))
+    ref, _ = p()
+    torch.cuda.synchronize()
+    ref = ref.clone()
+    for i in range(calls):
+        out, _ = p()
+        if i % 25 == 24 or i == calls - 1:
+            torch.cuda.synchronize()
+            assert p.status() == cuda_lib.QSA_OK, i
+            assert torch.equal(out, ref), i
+    assert torch.count_nonzero(_status_page(p.ws)) == 0
