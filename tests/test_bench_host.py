@@ -116,3 +116,26 @@ def test_executed_tensor_work_model():
     # tiles 28..31: chunks 0, 1 and the trailing chunk 3
     want2 = 28 + 4 * 3
     assert ex == want2 * per, (ex / per, want2)
+
+
+def test_cpu_sample_sized_past_the_fixed_cost(monkeypatch):
+    """The CPU baseline's sample lasts about the requested seconds even when a call
+    has a large fixed part: a fake oracle costs 2 s + 1 ms a row on a fake clock."""
+    w = W.small_variant(W.WORKLOADS["bf16_prefill_varlen_b8_s16384_leftpad"], seq=4096, batch=8, pad_max=200)
+    inp = W.make_inputs(w)
+    clock = [0.0]
+    runs = []
+
+    def fake_run(w_, inp_, rows=None, **kw):
+        n = sum(len(v) for v in rows.values())
+        runs.append(n)
+        clock[0] += 2.0 + 1e-3 * n
+
+    monkeypatch.setattr(oracle, "run", fake_run)
+    monkeypatch.setattr(bench.time, "perf_counter", lambda: clock[0])
+    r = bench.cpu_oracle_rate(w, inp, 15.0)
+    n_main = runs[-1]
+    assert runs[:2] == [32, 256]
+    # 2 s fixed + n_main ms ~= 15 s
+    assert abs((2.0 + 1e-3 * n_main) - 15.0) < 0.1, n_main
+    assert abs(r["value"] - n_main / (2.0 + 1e-3 * n_main)) < 1e-6
