@@ -128,6 +128,20 @@ def test_kernel_names_by_shape(qsa):
     assert qsa.qsa_attn_kernel_name(_cfg(qsa, d=256), qsa.QSA_DECODE) == "tcgen05 one-tile"
 
 
+def test_prefill_tensor_core_routing(qsa):
+    # a group size that divides the 128-row tile (up to 32, the config limit) and a block
+    # size that is a multiple of the 64-key half take the persistent tcgen05 kernel
+    for hq, hkv in [(2, 2), (4, 2), (8, 2), (16, 2), (32, 4), (32, 1), (64, 2)]:
+        for block in (64, 128, 192, 256):
+            c = _cfg(qsa, Hq=hq, Hkv=hkv, block=block, topk=4)
+            assert qsa.qsa_attn_kernel_name(c) == "tcgen05", (hq, hkv, block)
+    # a group of 12 (does not divide 128), a block of 32 keys, head_dim 64, fp32: CUDA cores
+    assert qsa.qsa_attn_kernel_name(_cfg(qsa, Hq=24, Hkv=2)) == "simt"
+    assert qsa.qsa_attn_kernel_name(_cfg(qsa, block=32)) == "simt"
+    assert qsa.qsa_attn_kernel_name(_cfg(qsa, d=64)) == "simt"
+    assert qsa.qsa_attn_kernel_name(_cfg(qsa, dtype="fp32")) == "simt"
+
+
 def test_offload_staging_size(qsa):
     # K and V of (k + 1) * B tokens per (sequence, KV head), then the remapped
     # selection and lengths, each section rounded up to 256 bytes
