@@ -57,6 +57,8 @@ def test_standalone_attention_shares_the_workspace(cuda_lib):
     dict(seq=1100, Hq=8, Hkv=2, block=64, topk=5),    # G = 4: k not a multiple of 4
     dict(seq=1100, Hq=16, Hkv=2, block=192, topk=3),  # a block size that is not a power of two
     dict(seq=2200, Hq=16, Hkv=2, block=256, topk=4),  # a block of two chunks
+    dict(seq=1100, Hq=32, Hkv=2, block=64, topk=8),   # G = 16: a softmax warp's rows are one token
+    dict(seq=1100, Hq=32, Hkv=1, block=128, topk=4),  # G = 32: 4 tokens a tile
 ])
 def test_tc_attention_unit_shapes_full_rows(cuda_lib, shape):
     """Unit shapes that take the builder's other paths (the lists loaded from global
